@@ -1,0 +1,103 @@
+"""ctypes front end of the fp64 oracle (test infrastructure only)."""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import numpy as np
+
+from .build import LIB, build
+
+_lib = None
+
+F16, BF16 = 0, 1
+
+
+def library_path() -> str:
+    return LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(LIB)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        lib.oracle_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I,
+                                      ctypes.c_double, I, P, P]
+        lib.oracle_decode.restype = I
+        lib.oracle_combine.argtypes = [P, P, I, ctypes.c_long, I, P, P]
+        lib.oracle_combine.restype = I
+        lib.oracle_f16_to_double.argtypes = [ctypes.c_uint16]
+        lib.oracle_f16_to_double.restype = ctypes.c_double
+        lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_double.restype = ctypes.c_double
+        _lib = lib
+    return _lib
+
+
+def _bits(x) -> np.ndarray:
+    """16-bit storage of a torch fp16/bf16 tensor or a numpy uint16 array."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch
+    assert x.dtype in (torch.float16, torch.bfloat16)
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def decode(q, k_cache, v_cache, block_table, cache_seqlens, *, Hkv: int,
+           page_size: int, dtype: str, scale: float, causal: bool,
+           max_pages_per_seq: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Exact attention in fp64.
+
+    q [B, q_len, Hq, D]; k_cache/v_cache [num_pages, page_size, Hkv, D]
+    (or [B, page_size, Hkv, D] when block_table is None); block_table
+    [B, max_pages_per_seq] int32 or None; cache_seqlens [B] int32.
+    Returns (out [B, q_len, Hq, D] float64, lse [B, Hq, q_len] float64).
+    """
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    B, q_len, Hq, D = qb.shape
+    L = np.ascontiguousarray(np.asarray(cache_seqlens, dtype=np.int32))
+    bt = None
+    mpps = 1
+    if block_table is not None:
+        bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+        mpps = bt.shape[1] if max_pages_per_seq is None else max_pages_per_seq
+    out = np.empty((B, q_len, Hq, D), dtype=np.float64)
+    lse = np.empty((B, Hq, q_len), dtype=np.float64)
+    rc = lib.oracle_decode(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(bt), _ptr(L), B, q_len, Hq,
+                           Hkv, D, page_size, mpps, BF16 if dtype == "bf16" else F16,
+                           float(scale), int(bool(causal)), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_decode: bad shape arguments")
+    return out, lse
+
+
+def combine(o_part: np.ndarray, lse_part: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Exact LSE merge.  o_part [S, rows, D], lse_part [S, rows] (float64)."""
+    lib = _load()
+    o_part = np.ascontiguousarray(o_part, dtype=np.float64)
+    lse_part = np.ascontiguousarray(lse_part, dtype=np.float64)
+    S, rows, D = o_part.shape
+    out = np.empty((rows, D), dtype=np.float64)
+    lse = np.empty((rows,), dtype=np.float64)
+    rc = lib.oracle_combine(_ptr(o_part), _ptr(lse_part), S, rows, D, _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_combine: bad shape arguments")
+    return out, lse
+
+
+def f16_to_double(bits: int) -> float:
+    return _load().oracle_f16_to_double(bits)
+
+
+def bf16_to_double(bits: int) -> float:
+    return _load().oracle_bf16_to_double(bits)
