@@ -1,0 +1,81 @@
+// Kernel argument blocks and host launch entry points (internal to libmxa).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "mxa.h"
+
+namespace mxa {
+
+// TMA descriptors of the K and V pools: 3-D maps {D, Hkv, pool tokens} with a
+// box of {64 elements, 1 head, box_tokens tokens} and 128-byte swizzle.
+struct alignas(64) TmapPair {
+  CUtensorMap k;
+  CUtensorMap v;
+};
+
+struct DecodeArgs {
+  const void *q;            // [B, q_len, Hq, D]
+  const int32_t *block_table;  // [B, mpps] (unused when contiguous)
+  const int32_t *seqlens;   // [B]
+  void *out;                // [B, q_len, Hq, D]
+  float *lse;               // [B, Hq, q_len] or null
+  int2 *meta;               // [units]: first and last CTA holding a piece of the unit
+  float *lse_part;          // [grid][2][16]
+  float *o_part;            // [grid][2][16][D]
+  int B, q_len, Hq, Hkv, G, M, RT;
+  int page_size;            // slots per page (row capacity when contiguous)
+  int mpps;                 // block-table row stride
+  int contiguous;
+  int max_seqlen_k;
+  int box_tokens;           // tokens per TMA box
+  float scale_log2;         // scale * log2(e)
+  int causal;
+  int schedule;             // mxa_schedule_t
+  int grid;
+  int splits;               // UNIFORM: splits per unit
+  int chunk_blocks;         // UNIFORM: blocks per split
+  int units;
+};
+
+struct MergeArgs {
+  const int2 *meta;
+  const float *lse_part;
+  const float *o_part;
+  void *out;
+  float *lse;
+  int q_len, Hq, Hkv, G, M, RT;
+  int grid;  // CTAs of the split kernel: metadata outside [0, grid) is ignored
+};
+
+// Everything launch_decode needs; pointers are device pointers.
+struct DecodeLaunch {
+  const void *q, *k_cache, *v_cache;
+  const int32_t *block_table, *seqlens;
+  void *out;
+  float *lse;
+  void *workspace;
+  mxa_decode_params_t p;
+  mxa_plan_t plan;
+  float scale;
+  int causal;
+};
+
+// Launch the split kernel and, when the plan needs it, the merge kernel.
+mxa_status_t launch_decode(const DecodeLaunch &L, cudaStream_t stream);
+
+// Launch the uniform-layout combine of mxa_combine().
+mxa_status_t launch_combine(const float *o_part, const float *lse_part, int num_splits, int B,
+                            int q_len, int Hq, int D, mxa_dtype_t dtype, void *out, float *lse,
+                            cudaStream_t stream);
+
+// Read (and optionally clear) the device-side failure record of the current device.
+mxa_status_t read_device_error(int reset, int *flags);
+
+// Multiprocessor count of the current device (cached per device).
+mxa_status_t current_sm_count(int *sm_count);
+
+}  // namespace mxa

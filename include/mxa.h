@@ -1,0 +1,223 @@
+/*
+ * mxa.h — C ABI of libmxa.so: exact paged grouped-query decode attention
+ * for NVIDIA B200 (sm_100a).
+ *
+ *   O = softmax(scale * Q K^T) V,   LSE = ln sum_j exp(scale * q . k_j)
+ *
+ * for decode and small-qLen (speculative / MTP) queries against a paged KV
+ * cache shared by groups of query heads.  The operation is the one stated in
+ * the "SmallQ FlashAttention (Vector)" README (section 接口, Interface:
+ * O = softmax(Q K^T / sqrt(headDim)) V with small qLen and long kvLen), on the
+ * paged KV cache of the "MXFlashAttn 1.4.0" project page (能力矩阵, the
+ * capability matrix: paged KV cache, FP16/BF16 forward, head_dim 64/128,
+ * GQA), computed with the online softmax of the "ops-transformer
+ * FlashAttention" walkthrough (section "FlashAttention 的数学细节"), the
+ * query-head packing and KV-axis split of "Flash-Attention GQA 性能调优:
+ * pack_gqa 与 num_splits 两个开关怎么选" (section "两个开关在 kernel 层面各做
+ * 了什么"), and a log-sum-exp merge of the split results.
+ *
+ * Conventions for every call:
+ *  - Pointers named as device pointers must point to device memory of the
+ *    current device, 16-byte aligned, in the layouts stated (row-major,
+ *    contiguous).  Scalars are passed by value.
+ *  - The library allocates no device memory and keeps no pointer after a
+ *    call returns.  The caller owns every buffer; scratch memory is the
+ *    caller's `workspace`, sized by mxa_plan().
+ *  - Launches are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL is the legacy default stream).  A returned status describes
+ *    argument checking and launch only; a device-side failure (a bounded
+ *    wait that ran out) is reported by mxa_device_error().
+ *  - No call aborts the process, traps the GPU or falls back to another
+ *    implementation: an unsupported shape is refused with a status code.
+ */
+#ifndef MXA_H_
+#define MXA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MXA_API __attribute__((visibility("default")))
+#else
+#define MXA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes (integer codes, in the style of the aclnn
+ * ACLNN_ERR_PARAM_INVALID family in "MixedQuantSparseFlashMlaMetadata
+ * 算子解析", section 参数说明 / 约束说明). */
+typedef enum {
+  MXA_OK = 0,
+  MXA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad shape or stride */
+  MXA_ERR_UNSUPPORTED = 2,   /* a shape the kernels do not implement (e.g. D not 64/128) */
+  MXA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than mxa_plan() says */
+  MXA_ERR_CUDA = 4,          /* a CUDA runtime call failed (no device, launch error) */
+  MXA_ERR_TIMEOUT = 5        /* a device-side bounded wait ran out (see mxa_device_error) */
+} mxa_status_t;
+
+typedef enum { MXA_F16 = 0, MXA_BF16 = 1 } mxa_dtype_t;
+
+/* Work schedules of the split kernel.
+ * UNIFORM:  every (batch row, KV head, row tile) unit has its KV axis cut at
+ *           multiples of one chunk, chunk = ceil(max_seqlen_k / num_splits)
+ *           tokens rounded up to the pipeline block; grid = units * num_splits.
+ *           num_splits = 1 means one CTA per unit and no combine pass.
+ * BALANCED: the KV blocks of all units, laid end to end (unit-major), are
+ *           divided into `grid` equal contiguous ranges, one per CTA; a unit
+ *           that straddles ranges is merged by the combine pass.  Every CTA
+ *           streams the same number of KV bytes however ragged the lengths
+ *           are (a length-aware split in the spirit of the cost-balanced
+ *           core assignment of "MixedQuantSparseFlashMlaMetadata 算子解析",
+ *           section 源码级原理). */
+typedef enum { MXA_SCHED_UNIFORM = 0, MXA_SCHED_BALANCED = 1 } mxa_schedule_t;
+
+/* Problem shape.
+ *   q            [B, q_len, Hq, D]                 dtype
+ *   k/v cache    [num_pages, page_size, Hkv, D]     dtype   (paged)
+ *                [B, page_size, Hkv, D]             dtype   (contiguous: block_table == NULL,
+ *                                                            num_pages == B, page_size = row capacity)
+ *   block_table  [B, max_pages_per_seq] int32: page id of logical page p of row b
+ *   cache_seqlens[B] int32: number of valid keys L_b, 0 <= L_b <= max_seqlen_k
+ *   out          [B, q_len, Hq, D]                 dtype
+ *   lse          [B, Hq, q_len]                    float32, natural log
+ * Query head h reads KV head h / (Hq / Hkv).
+ * max_seqlen_k is an upper bound on every L_b known on the host; it sizes
+ * the uniform split without reading device memory. */
+typedef struct {
+  int B, q_len, Hq, Hkv, D;
+  int num_pages, page_size;
+  int max_pages_per_seq;
+  int max_seqlen_k;
+  mxa_dtype_t dtype;
+} mxa_decode_params_t;
+
+/* A resolved execution plan (the host half of the two-phase call: plan,
+ * then run; compare the GetWorkspaceSize-then-execute pattern of the aclnn
+ * API in the "SmallQ FlashAttention (Vector)" README, section aclnn API 调用). */
+typedef struct {
+  int num_splits;        /* splits per unit (>= 1); BALANCED: grid / units */
+  int schedule;          /* mxa_schedule_t */
+  int grid;              /* CTAs of the split kernel */
+  int units;             /* B * Hkv * ceil(q_len * G / 16) */
+  int rows_per_tile;     /* packed query rows per tile (16) */
+  int block_tokens;      /* KV tokens per pipeline stage */
+  int ctas_per_sm;       /* resident CTAs per SM the plan assumed */
+  int sm_count;          /* SMs the plan assumed */
+  int needs_combine;     /* 1 if a combine pass follows the split kernel */
+  size_t workspace_bytes;/* device scratch the run needs (0 if none) */
+} mxa_plan_t;
+
+/* Text for a status code; never NULL. */
+MXA_API const char *mxa_status_string(mxa_status_t status);
+
+/* The GQA packing rule of "Flash-Attention GQA 性能调优", section
+ * "pack_gqa 怎么选": varlen queries always pack; otherwise pack iff the row
+ * efficiency without packing, seqlen_q / round_up(seqlen_q, block_m), is
+ * below 0.9 times the efficiency with packing,
+ * seqlen_q*qpk / round_up(seqlen_q*qpk, block_m).  Returns 1 (pack) or 0.
+ * Pure host function.  The kernels here always pack; this rule is exported
+ * so callers and tests can see that it agrees for every decode shape. */
+MXA_API int mxa_should_pack_gqa(int varlen_q, int seqlen_q, int qhead_per_khead, int block_m);
+
+/* The num_splits rule of the same page, section "num_splits 怎么选":
+ *  (i)  if the tiles (batch x KV heads x query tiles) reach 80% of the SM
+ *       count, use 1 split (except a non-causal problem whose single KV head
+ *       exceeds the ~50 MB L2 figure with several query tiles, which splits
+ *       by the ratio of KV-head bytes to that figure);
+ *  (ii) if the KV axis has at most 4 blocks of block_n tokens, use 1;
+ *  (iii) otherwise take, over s = 1..max_splits, the wave efficiency
+ *       n_waves / ceil(n_waves) with n_waves = tiles * s / slots, and return
+ *       the smallest s whose efficiency is at least 85% of the best.
+ * `slots` is the number of CTAs one wave holds (SMs x resident CTAs per SM);
+ * `kv_head_bytes` is the K+V bytes of one KV head of one sequence.
+ * Pure host function; returns >= 1, or 0 on a bad argument. */
+MXA_API int mxa_num_splits_heuristic(int tiles, int sm_count, int slots, int num_n_blocks,
+                             int max_splits, int causal, int num_m_blocks,
+                             double kv_head_bytes);
+
+/* Resolve a plan for `params`.
+ *   num_splits > 0 : UNIFORM schedule with that many splits per unit.
+ *   num_splits == 0: automatic: s from mxa_num_splits_heuristic, BALANCED
+ *                    schedule with grid = units * s.
+ *   sm_count > 0   : plan for that many SMs (pure host computation);
+ *   sm_count <= 0  : query the current CUDA device (MXA_ERR_CUDA without one).
+ * Errors: MXA_ERR_INVALID_ARG for a NULL pointer or an inconsistent shape
+ * (B < 0, q_len < 1, Hq % Hkv != 0, page_size < 1, ...);
+ * MXA_ERR_UNSUPPORTED for D not in {64, 128} or sizes past the int32
+ * index range.  The page size is checked by the run calls, which know
+ * whether the cache is paged: a paged cache needs page_size to divide the
+ * stage of block_tokens tokens and be a multiple of 8, or to be a multiple
+ * of block_tokens (else MXA_ERR_UNSUPPORTED); a contiguous cache takes any
+ * row capacity >= max_seqlen_k. */
+MXA_API mxa_status_t mxa_plan(const mxa_decode_params_t *params, int num_splits, int sm_count,
+                      mxa_plan_t *plan);
+
+/* A BALANCED plan over an explicit number of CTAs (grid >= 1), for tuning
+ * the split and for tests: the same as mxa_plan's automatic plan with its
+ * grid replaced.  Pure host computation apart from sm_count <= 0, which
+ * queries the current device.  Errors as mxa_plan; MXA_ERR_UNSUPPORTED if
+ * B exceeds the 16384 rows the balanced prologue scans. */
+MXA_API mxa_status_t mxa_plan_balanced(const mxa_decode_params_t *params, int grid, int sm_count,
+                                       mxa_plan_t *plan);
+
+/* Decode attention, one call: plan (num_splits as in mxa_plan, on the
+ * current device) and run.
+ *   q, k_cache, v_cache, block_table, cache_seqlens : device, read only
+ *   block_table may be NULL for a contiguous cache (see mxa_decode_params_t).
+ *   scale      : multiplies Q K^T (usually 1/sqrt(D))
+ *   causal     : 0 = every query row sees all L_b keys; 1 = query t (0-based)
+ *                sees the first L_b - q_len + t + 1 keys (the draft tokens are
+ *                the last q_len entries of the cache; the RightDownCausal mask
+ *                of "MixedQuantSparseFlashMlaMetadata 算子解析", 参数说明)
+ *   workspace  : device scratch of at least plan.workspace_bytes (may be NULL
+ *                when that is 0); contents on entry are ignored
+ *   out        : device [B, q_len, Hq, D] dtype (written in full)
+ *   lse        : device [B, Hq, q_len] float32, or NULL to skip
+ * A row that sees no key gets O = 0 and LSE = -inf.
+ * Returns MXA_ERR_WORKSPACE if the workspace is missing or too small. */
+MXA_API mxa_status_t mxa_decode_fwd(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *block_table, const int32_t *cache_seqlens,
+                            const mxa_decode_params_t *params, float scale, int causal,
+                            int num_splits, void *workspace, size_t workspace_bytes,
+                            void *out, float *lse, void *stream);
+
+/* As mxa_decode_fwd, but run a plan the caller resolved (or built) before:
+ * the second phase of the two-phase call.  The plan is validated against
+ * `params` (schedule, grid >= 1, units, block_tokens); a BALANCED plan may
+ * use any grid >= 1. */
+MXA_API mxa_status_t mxa_decode_fwd_with_plan(const void *q, const void *k_cache, const void *v_cache,
+                                      const int32_t *block_table, const int32_t *cache_seqlens,
+                                      const mxa_decode_params_t *params, float scale, int causal,
+                                      const mxa_plan_t *plan, void *workspace,
+                                      size_t workspace_bytes, void *out, float *lse,
+                                      void *stream);
+
+/* Merge split results with the log-sum-exp identity (the reduce that
+ * follows a KV-axis split, "Flash-Attention GQA 性能调优", section
+ * "两个开关在 kernel 层面各做了什么"):
+ *   LSE = ln sum_s exp(lse_s),   O = sum_s exp(lse_s - LSE) O_s
+ * with the largest lse_s subtracted for stability; splits with lse_s = -inf
+ * carry no weight; if all are -inf, O = 0 and LSE = -inf.
+ *   o_part   device [num_splits, B, q_len, Hq, D] float32 (each O_s normalised)
+ *   lse_part device [num_splits, B, Hq, q_len]    float32 (natural log)
+ *   out      device [B, q_len, Hq, D] dtype
+ *   lse      device [B, Hq, q_len] float32, or NULL
+ * D must be a multiple of 4 and at most 512. */
+MXA_API mxa_status_t mxa_combine(const float *o_part, const float *lse_part, int num_splits, int B,
+                         int q_len, int Hq, int D, mxa_dtype_t dtype, void *out, float *lse,
+                         void *stream);
+
+/* Synchronise the current device and report whether any kernel of this
+ * library recorded a device-side failure (a bounded wait that ran out) since
+ * the last reset: MXA_OK or MXA_ERR_TIMEOUT (MXA_ERR_CUDA if the device or
+ * the synchronisation itself failed).  reset != 0 clears the record. */
+MXA_API mxa_status_t mxa_device_error(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXA_H_ */

@@ -1,0 +1,229 @@
+"""GPU parity: the CUDA path of libmxa.so against the fp64 oracle, element
+by element, on the same seeded inputs.
+
+Covers the five decode workloads at their full sizes in the launch
+configuration the benchmark times, the split sweeps, both schedules with
+many grid sizes, ragged and edge lengths, every supported page size and the
+contiguous layout, grouped-query ratios and query lengths (causal and not),
+rows that see no key, garbage (NaN) in unused cache slots, the public
+combine, determinism and the device failure record.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from decode_attention_packed_b200.workloads import WORKLOADS, Workload, make_inputs
+from tests.tolerance import assert_lse_close, assert_out_close
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from decode_attention_packed_b200 import mxa
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _needs_cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def run_oracle(inp):
+    w = inp.w
+    return oracle.decode(inp.q, inp.k_cache, inp.v_cache, inp.block_table, inp.cache_seqlens,
+                         Hkv=w.Hkv, page_size=inp.page_size, dtype=w.dtype, scale=w.scale,
+                         causal=w.causal)
+
+
+def to_dev(inp):
+    d = "cuda"
+    bt = None if inp.block_table is None else inp.block_table.to(d)
+    return inp.q.to(d), inp.k_cache.to(d), inp.v_cache.to(d), bt, inp.cache_seqlens.to(d)
+
+
+def run_gpu(inp, num_splits=0, plan=None, dev=None, return_lse=True):
+    q, k, v, bt, sl = dev if dev is not None else to_dev(inp)
+    prep = mxa.prepare(q, k, bt, max_seqlen_k=inp.max_seqlen_k, num_splits=num_splits, plan=plan)
+    out, lse = mxa.decode(q, k, v, bt, sl, scale=inp.w.scale, causal=inp.w.causal, prepared=prep,
+                          return_lse=return_lse)
+    torch.cuda.synchronize()
+    assert mxa.mxa_device_error(True) == mxa.MXA_OK
+    return out.cpu(), (None if lse is None else lse.cpu()), prep.plan
+
+
+def check(inp, out, lse, ref=None):
+    ro, rl = run_oracle(inp) if ref is None else ref
+    err = assert_out_close(out, ro, inp.w.dtype)
+    if lse is not None:
+        assert_lse_close(lse, rl)
+    return err
+
+
+_cache = {}
+
+
+def full(i):
+    if i not in _cache:
+        inp = make_inputs(WORKLOADS[i])
+        _cache[i] = (inp, run_oracle(inp), to_dev(inp))
+    return _cache[i]
+
+
+# --------------------------------------------------------------------------
+# the five workloads at full size
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("i", range(len(WORKLOADS)))
+def test_workload_full_size(i):
+    inp, ref, dev = full(i)
+    out, lse, plan = run_gpu(inp, num_splits=inp.w.num_splits, dev=dev)
+    err = check(inp, out, lse, ref)
+    print(f"{inp.w.name}: plan={plan.as_dict()} max|err|={err:.3e}")
+
+
+@pytest.mark.parametrize("s", [1, 2, 4, 8, 16])
+def test_long_context_split_sweep(s):
+    inp, ref, dev = full(3)
+    out, lse, plan = run_gpu(inp, num_splits=s, dev=dev)
+    assert plan.schedule == mxa.MXA_SCHED_UNIFORM and plan.grid == 16 * s
+    check(inp, out, lse, ref)
+
+
+@pytest.mark.parametrize("s", [1, 3, 8])
+def test_ragged_uniform_splits(s):
+    inp, ref, dev = full(1)
+    out, lse, _ = run_gpu(inp, num_splits=s, dev=dev)
+    check(inp, out, lse, ref)
+
+
+@pytest.mark.parametrize("grid", [1, 2, 7, 148, 296, 1000, 5000])
+def test_ragged_balanced_grids(grid):
+    inp, ref, dev = full(4)
+    q, k, v, bt, sl = dev
+    plan = mxa.mxa_plan_balanced(mxa.params_for(q, k, bt, inp.max_seqlen_k), grid)
+    assert plan.grid == grid and plan.schedule == mxa.MXA_SCHED_BALANCED
+    out, lse, _ = run_gpu(inp, plan=plan, dev=dev)
+    check(inp, out, lse, ref)
+
+
+# --------------------------------------------------------------------------
+# shapes and edges at sizes the oracle finishes in seconds
+# --------------------------------------------------------------------------
+
+EDGE_LENGTHS = [0, 1, 2, 15, 16, 17, 63, 64, 65, 127, 128, 129, 255, 257, 1023, 1025, 1500, 3000, 4096]
+
+
+def wl(**kw):
+    base = dict(name="case", B=len(EDGE_LENGTHS), q_len=1, Hq=8, Hkv=2, D=128, dtype="bf16",
+                page_size=16, causal=False, lengths="list:" + ",".join(map(str, EDGE_LENGTHS)), seed=11)
+    base.update(kw)
+    return Workload(**base)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("num_splits", [0, 1, 3])
+def test_edge_lengths(D, dtype, num_splits):
+    inp = make_inputs(wl(D=D, dtype=dtype))
+    out, lse, _ = run_gpu(inp, num_splits=num_splits)
+    check(inp, out, lse)
+    assert (out[0] == 0).all() and torch.isneginf(lse[0]).all()   # the L = 0 row
+
+
+@pytest.mark.parametrize("page", [0, 8, 16, 32, 64, 128, 256, 192])
+@pytest.mark.parametrize("D", [64, 128])
+def test_page_sizes(page, D):
+    if page == 192 and D == 64:
+        pytest.skip("192 neither divides nor is a multiple of the 128-key stage")
+    inp = make_inputs(wl(page_size=page, D=D, lengths="list:1,100,700,1030,2049", B=5, seed=page + D))
+    for s in (0, 2):
+        out, lse, _ = run_gpu(inp, num_splits=s)
+        check(inp, out, lse)
+
+
+def test_page_size_not_tiling_is_refused():
+    inp = make_inputs(wl(page_size=24, lengths="list:50", B=1))
+    with pytest.raises(mxa.MxaError) as e:
+        run_gpu(inp)
+    assert e.value.code == mxa.MXA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("q_len", [1, 2, 4, 8])
+@pytest.mark.parametrize("causal", [False, True])
+def test_groups_and_query_lengths(G, q_len, causal):
+    inp = make_inputs(wl(Hq=2 * G, Hkv=2, q_len=q_len, causal=causal, D=64 if G % 2 else 128,
+                         lengths="list:3,9,130,1025", B=4, page_size=32, seed=G * 10 + q_len))
+    for s in (0, 1):
+        out, lse, plan = run_gpu(inp, num_splits=s)
+        assert plan.units == 4 * 2 * math.ceil(q_len * G / 16)
+        check(inp, out, lse)
+
+
+def test_causal_rows_with_no_key():
+    inp = make_inputs(wl(q_len=8, causal=True, Hq=16, Hkv=4, lengths="list:1,3,7,8,9", B=5, seed=5))
+    out, lse, _ = run_gpu(inp)
+    check(inp, out, lse)
+    assert torch.isneginf(lse[0, :, :7]).all() and (out[0, :7] == 0).all()
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_nan_in_unused_cache_slots(dtype):
+    """Slots past L_b in a row's last page and pages no row uses hold NaN:
+    the result is the same as with clean memory."""
+    w = wl(dtype=dtype, lengths="list:5,33,70,0", B=4, page_size=32, seed=21)
+    inp = make_inputs(w)
+    ref = run_oracle(inp)
+    extra = torch.full((3,) + tuple(inp.k_cache.shape[1:]), float("nan"), dtype=inp.k_cache.dtype)
+    inp.k_cache = torch.cat([inp.k_cache, extra])
+    inp.v_cache = torch.cat([inp.v_cache, extra.clone()])
+    for b, L in enumerate(inp.cache_seqlens.tolist()):
+        if L % 32:
+            pg = int(inp.block_table[b, L // 32])
+            inp.k_cache[pg, L % 32:] = float("nan")
+            inp.v_cache[pg, L % 32:] = float("nan")
+    for s in (0, 1, 2):
+        out, lse, _ = run_gpu(inp, num_splits=s)
+        check(inp, out, lse, ref)
+
+
+def test_contiguous_with_spare_capacity():
+    inp = make_inputs(wl(page_size=0, lengths="list:1,77,300,0,513", B=5, seed=3), max_seqlen_k=600)
+    inp.v_cache[:, 513:] = float("nan")   # capacity past every row's length
+    for s in (0, 1, 4):
+        out, lse, _ = run_gpu(inp, num_splits=s)
+        check(inp, out, lse)
+
+
+def test_lse_is_optional_and_runs_are_deterministic():
+    inp, ref, dev = full(1)
+    o1, _, _ = run_gpu(inp, dev=dev, return_lse=False)
+    o2, l2, _ = run_gpu(inp, dev=dev)
+    assert torch.equal(o1, o2)
+    check(inp, o2, l2, ref)
+
+
+# --------------------------------------------------------------------------
+# public combine
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_combine_matches_exact_merge(dtype):
+    rng = np.random.default_rng(9)
+    S, B, q_len, Hq, D = 5, 3, 2, 4, 64
+    o = rng.standard_normal((S, B, q_len, Hq, D)).astype(np.float32)
+    lse = (rng.standard_normal((S, B, Hq, q_len)) * 4).astype(np.float32)
+    lse[1, 0] = -np.inf                 # an empty split
+    lse[:, 2, 1, 0] = -np.inf           # a row with no key in any split
+    rows_o = o.transpose(0, 1, 2, 3, 4).reshape(S, -1, D)
+    rows_l = lse.transpose(0, 1, 3, 2).reshape(S, -1)    # [S, B*q_len*Hq] in (b, t, h) order
+    ro, rl = oracle.combine(rows_o.astype(np.float64), rows_l.astype(np.float64))
+    out = torch.empty((B, q_len, Hq, D), dtype=torch.bfloat16 if dtype == "bf16" else torch.float16,
+                      device="cuda")
+    lse_out = torch.empty((B, Hq, q_len), dtype=torch.float32, device="cuda")
+    mxa.mxa_combine(torch.from_numpy(o).cuda(), torch.from_numpy(lse).cuda(), out, lse_out)
+    torch.cuda.synchronize()
+    assert_out_close(out.cpu(), ro.reshape(B, q_len, Hq, D), dtype)
+    assert_lse_close(lse_out.cpu(), rl.reshape(B, q_len, Hq).transpose(0, 2, 1))

@@ -1,0 +1,182 @@
+"""Host-side checks of libmxa.so that need no GPU: the library loads and
+exports every symbol include/mxa.h declares, the planner and the packing and
+split rules follow the pages' worked cases, and bad arguments are refused
+with status codes before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from decode_attention_packed_b200 import mxa
+from decode_attention_packed_b200.mxa import (MXA_ERR_INVALID_ARG, MXA_ERR_UNSUPPORTED,
+                                              MXA_ERR_WORKSPACE, MXA_OK, MXA_SCHED_BALANCED,
+                                              MXA_SCHED_UNIFORM, mxa_decode_params_t, mxa_plan_t)
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GOLDEN = os.path.join(ROOT, "tests", "golden", "heuristics_pack_gqa_num_splits.txt")
+
+
+def header_symbols():
+    text = open(os.path.join(ROOT, "include", "mxa.h")).read()
+    return sorted(set(re.findall(r"MXA_API\s+[\w\s\*]*?\b(mxa_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = header_symbols()
+    assert len(names) >= 8, names
+    lib = ctypes.CDLL(mxa.LIBRARY)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/mxa.h but not exported"
+    assert sorted(mxa.EXPORTED) == names
+
+
+def test_status_strings():
+    for code in range(6):
+        assert mxa.mxa_status_string(code).startswith("MXA_")
+    assert "UNKNOWN" in mxa.mxa_status_string(99)
+
+
+def golden_rows(kind):
+    for line in open(GOLDEN):
+        line = line.split("#")[0].split()
+        if line and line[0] == kind:
+            yield [int(x) for x in line[1:]]
+
+
+def test_pack_gqa_rule_worked_cases():
+    rows = list(golden_rows("pack"))
+    assert rows
+    for varlen, seqlen_q, qpk, block_m, expect in rows:
+        assert mxa.mxa_should_pack_gqa(varlen, seqlen_q, qpk, block_m) == expect
+
+
+@pytest.mark.parametrize("q_len,G", [(1, 2), (1, 4), (1, 8), (4, 8), (8, 2), (2, 16)])
+def test_pack_gqa_holds_for_every_decode_shape(q_len, G):
+    """The kernels always pack; the rule agrees for small q_len (block_m 16)."""
+    assert mxa.mxa_should_pack_gqa(0, q_len, G, 16) == 1
+
+
+def test_num_splits_rule_worked_cases():
+    rows = list(golden_rows("splits"))
+    assert rows
+    for batch, hkv, m_rows, seqlen_k, block_m, block_n, sms, max_splits, expect in rows:
+        tiles = batch * hkv * ((m_rows + block_m - 1) // block_m)
+        n_blocks = (seqlen_k + block_n - 1) // block_n
+        got = mxa.mxa_num_splits_heuristic(tiles, sms, sms, n_blocks, max_splits, 0, 1,
+                                           seqlen_k * 128 * 4.0)
+        assert got == expect, (batch, got, expect)
+
+
+def test_num_splits_wave_efficiency():
+    # 16 tiles on 148 slots: eff(s) = 16s/148 / ceil(16s/148); best 1.0 (s = 37);
+    # smallest s with eff >= 0.85 is 8 (128/148 = 0.865; 7 gives 0.757)
+    assert mxa.mxa_num_splits_heuristic(16, 148, 148, 128, 128, 0, 1, 1e6) == 8
+    # the same on 296 slots (two CTAs per SM): 16 (256/296 = 0.865)
+    assert mxa.mxa_num_splits_heuristic(16, 148, 296, 128, 128, 0, 1, 1e6) == 16
+    # enough tiles: one split
+    assert mxa.mxa_num_splits_heuristic(256, 148, 296, 64, 64, 0, 1, 1e6) == 1
+    # the large-KV-head exception: non-causal, several query tiles
+    big = 200 * 1024 * 1024
+    assert mxa.mxa_num_splits_heuristic(256, 148, 296, 4096, 128, 0, 4, big) == 4
+    assert mxa.mxa_num_splits_heuristic(256, 148, 296, 4096, 128, 1, 4, big) == 1
+    assert mxa.mxa_num_splits_heuristic(0, 148, 296, 4096, 128, 0, 1, 1.0) == 0
+
+
+def params(**kw):
+    base = dict(B=2, q_len=1, Hq=64, Hkv=8, D=128, num_pages=512, page_size=64,
+                max_pages_per_seq=256, max_seqlen_k=16384, dtype=mxa.MXA_BF16)
+    base.update(kw)
+    return mxa_decode_params_t(*[base[f] for f, _ in mxa_decode_params_t._fields_])
+
+
+def test_plan_long_context_split():
+    plan = mxa.mxa_plan(params(), 0, sm_count=148)
+    assert plan.schedule == MXA_SCHED_BALANCED
+    assert plan.units == 16 and plan.num_splits == 16 and plan.grid == 256
+    assert plan.ctas_per_sm == 2 and plan.block_tokens == 64
+    assert plan.needs_combine == 1 and plan.workspace_bytes > 0
+
+
+def test_plan_uniform_and_row_tiles():
+    plan = mxa.mxa_plan(params(B=16, q_len=4, Hq=32), 4, sm_count=148)
+    assert plan.schedule == MXA_SCHED_UNIFORM and plan.grid == 16 * 8 * 4
+    p1 = mxa.mxa_plan(params(B=16, q_len=4, Hq=32), 1, sm_count=148)
+    assert p1.needs_combine == 0 and p1.workspace_bytes == 0
+    # 8 query heads per KV head x 4 tokens = 32 packed rows = 2 row tiles
+    p2 = mxa.mxa_plan(params(B=3, q_len=4, Hq=64), 1, sm_count=148)
+    assert p2.units == 3 * 8 * 2
+    # D = 64 stages carry 128 keys
+    assert mxa.mxa_plan(params(D=64), 1, sm_count=148).block_tokens == 128
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=96), MXA_ERR_UNSUPPORTED),
+    (dict(D=256), MXA_ERR_UNSUPPORTED),
+    (dict(Hq=12, Hkv=8), MXA_ERR_INVALID_ARG),
+    (dict(q_len=0), MXA_ERR_INVALID_ARG),
+    (dict(B=-1), MXA_ERR_INVALID_ARG),
+    (dict(page_size=0), MXA_ERR_INVALID_ARG),
+    (dict(dtype=7), MXA_ERR_INVALID_ARG),
+])
+def test_plan_refuses_bad_shapes(kw, code):
+    plan = mxa_plan_t()
+    p = params(**kw)
+    assert mxa._lib.mxa_plan(ctypes.byref(p), 0, 148, ctypes.byref(plan)) == code
+
+
+def _run_with_plan(p, plan, *, q=1, k=1, v=1, bt=1, sl=1, out=1, ws=None, ws_bytes=0, lse=None,
+                   scale=0.125, causal=0):
+    f = lambda x: None if x is None else ctypes.c_void_p(x * 4096)
+    return mxa._lib.mxa_decode_fwd_with_plan(f(q), f(k), f(v), f(bt), f(sl), ctypes.byref(p),
+                                             scale, causal, ctypes.byref(plan), f(ws), ws_bytes,
+                                             f(out), f(lse), None)
+
+
+def test_run_refuses_bad_arguments_before_launch():
+    p = params()
+    plan = mxa.mxa_plan(p, 0, sm_count=148)
+    assert _run_with_plan(p, plan, q=None) == MXA_ERR_INVALID_ARG
+    assert _run_with_plan(p, plan, out=None) == MXA_ERR_INVALID_ARG
+    assert _run_with_plan(p, plan, sl=None) == MXA_ERR_INVALID_ARG
+    assert _run_with_plan(p, plan, ws=None) == MXA_ERR_WORKSPACE
+    assert _run_with_plan(p, plan, ws=1, ws_bytes=plan.workspace_bytes - 1) == MXA_ERR_WORKSPACE
+    assert _run_with_plan(p, plan, scale=float("nan")) == MXA_ERR_INVALID_ARG
+    assert _run_with_plan(p, plan, causal=2) == MXA_ERR_INVALID_ARG
+    # misaligned pointer
+    f = lambda x: ctypes.c_void_p(x)
+    assert mxa._lib.mxa_decode_fwd_with_plan(f(4096 + 2), f(4096), f(4096), f(4096), f(4096),
+                                             ctypes.byref(p), 0.1, 0, ctypes.byref(plan), f(4096),
+                                             plan.workspace_bytes, f(4096), None, None) == MXA_ERR_INVALID_ARG
+    # a page size the gather does not tile (paged) ...
+    p12 = params(page_size=12, max_pages_per_seq=2048)
+    assert _run_with_plan(p12, mxa.mxa_plan(p12, 1, sm_count=148)) == MXA_ERR_UNSUPPORTED
+    # ... block table too narrow for max_seqlen_k
+    pn = params(max_pages_per_seq=8)
+    assert _run_with_plan(pn, mxa.mxa_plan(pn, 1, sm_count=148)) == MXA_ERR_INVALID_ARG
+    # a uniform plan whose grid does not match units x splits
+    bad = mxa.mxa_plan(p, 2, sm_count=148)
+    bad.grid += 1
+    assert _run_with_plan(p, bad, ws=1, ws_bytes=1 << 30) == MXA_ERR_INVALID_ARG
+    # nothing to do for B = 0
+    p0 = params(B=0)
+    assert _run_with_plan(p0, mxa.mxa_plan(p0, 1, sm_count=148)) == MXA_OK
+
+
+def test_combine_refuses_bad_arguments():
+    f = lambda x: None if x is None else ctypes.c_void_p(x * 4096)
+    c = mxa._lib.mxa_combine
+    assert c(f(1), f(1), 0, 2, 1, 4, 64, 0, f(1), None, None) == MXA_ERR_INVALID_ARG
+    assert c(f(1), f(1), 2, 2, 1, 4, 66, 0, f(1), None, None) == MXA_ERR_INVALID_ARG
+    assert c(None, f(1), 2, 2, 1, 4, 64, 0, f(1), None, None) == MXA_ERR_INVALID_ARG
+    assert c(f(1), f(1), 2, 0, 1, 4, 64, 0, f(1), None, None) == MXA_OK
+
+
+def test_params_from_tensors():
+    q = torch.empty(3, 2, 8, 64, dtype=torch.float16)
+    k = torch.empty(40, 16, 2, 64, dtype=torch.float16)
+    bt = torch.zeros(3, 7, dtype=torch.int32)
+    p = mxa.params_for(q, k, bt)
+    assert (p.B, p.q_len, p.Hq, p.Hkv, p.D, p.num_pages, p.page_size, p.max_pages_per_seq,
+            p.max_seqlen_k, p.dtype) == (3, 2, 8, 2, 64, 40, 16, 7, 112, mxa.MXA_F16)
