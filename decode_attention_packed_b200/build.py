@@ -15,7 +15,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libmxa.so")
-SOURCES = [os.path.join(CSRC, "mxa_kernels.cu"), os.path.join(CSRC, "mxa_api.cpp")]
+SOURCES = [os.path.join(CSRC, "mxa_kernels.cu"), os.path.join(CSRC, "mxa_api.cpp"),
+           os.path.join(CSRC, "mxa_noalloc.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("mxa_config.h", "mxa_device.cuh", "mxa_launch.h")] + \
     [os.path.join(INCLUDE, "mxa.h")]
 

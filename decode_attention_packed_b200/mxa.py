@@ -29,7 +29,8 @@ MXA_SCHED_UNIFORM, MXA_SCHED_BALANCED = 0, 1
 
 EXPORTED = ("mxa_status_string", "mxa_should_pack_gqa", "mxa_num_splits_heuristic", "mxa_plan",
             "mxa_plan_balanced",
-            "mxa_decode_fwd", "mxa_decode_fwd_with_plan", "mxa_combine", "mxa_device_error")
+            "mxa_decode_fwd", "mxa_decode_fwd_with_plan", "mxa_combine", "mxa_device_error",
+            "mxa_decode_fwd_noalloc")
 
 
 class mxa_decode_params_t(ctypes.Structure):
@@ -69,6 +70,9 @@ _lib.mxa_decode_fwd_with_plan.argtypes = [_P, _P, _P, _P, _P, ctypes.POINTER(mxa
                                           ctypes.c_float, _I, ctypes.POINTER(mxa_plan_t), _P,
                                           ctypes.c_size_t, _P, _P, _P]
 _lib.mxa_decode_fwd_with_plan.restype = _I
+_lib.mxa_decode_fwd_noalloc.argtypes = [_P, _P, _P, _P, _P, ctypes.POINTER(mxa_decode_params_t),
+                                        ctypes.c_float, _I, _I, _P, _P, _P]
+_lib.mxa_decode_fwd_noalloc.restype = _I
 _lib.mxa_combine.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]
 _lib.mxa_combine.restype = _I
 _lib.mxa_device_error.argtypes = [_I]
@@ -144,6 +148,18 @@ def mxa_decode_fwd_with_plan(q, k_cache, v_cache, block_table, cache_seqlens, pa
                                          int(causal), ctypes.byref(plan), _ptr(workspace), ws_bytes,
                                          _ptr(out), _ptr(lse), _stream(stream)),
            "mxa_decode_fwd_with_plan")
+
+
+def mxa_decode_fwd_noalloc(q, k_cache, v_cache, block_table, cache_seqlens, params, scale, causal,
+                           num_splits, out, lse, stream=None) -> None:
+    """Decode with the library's fixed 16 MiB scratch array instead of a
+    workspace, for callers that cannot allocate device memory (see
+    include/mxa.h: first call per device before any stream capture; calls
+    that overlap on the GPU race on the shared array)."""
+    _check(_lib.mxa_decode_fwd_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                       _ptr(cache_seqlens), ctypes.byref(params), float(scale),
+                                       int(causal), int(num_splits), _ptr(out), _ptr(lse),
+                                       _stream(stream)), "mxa_decode_fwd_noalloc")
 
 
 def mxa_combine(o_part, lse_part, out, lse=None, stream=None) -> None:

@@ -195,6 +195,35 @@ MXA_API mxa_status_t mxa_decode_fwd_with_plan(const void *q, const void *k_cache
                                       size_t workspace_bytes, void *out, float *lse,
                                       void *stream);
 
+/* Decode without any device allocation, for callers that cannot allocate.
+ * (An addition of this library; the source pages have no counterpart.)
+ *
+ * Some callers cannot call cudaMalloc at the point where they run a decode
+ * step: an engine that reserves all device memory at start-up and forbids
+ * allocation inside its step loop, a plugin living under another framework's
+ * memory manager, or a latency-critical loop where an allocation call could
+ * synchronise the device.  This call is mxa_decode_fwd without the workspace
+ * arguments: it plans the same way (num_splits as in mxa_plan) and runs the
+ * same kernels, but keeps the split results in one fixed 16 MiB array inside
+ * the library.  It calls no allocator at all.
+ *  - The array is part of the library's device image: every GPU that loads
+ *    the library holds those 16 MiB until the process exits.
+ *  - A plan that needs more scratch than 16 MiB is refused with
+ *    MXA_ERR_WORKSPACE (use mxa_decode_fwd with your own workspace then).
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make
+ *    that first call before any stream capture.
+ *  - Every call on a device shares the one array, which keeps whatever the
+ *    last call left in it.  Nothing in it needs to start at zero: each call
+ *    rewrites every entry it later reads.  Calls whose kernels overlap on the
+ *    GPU (other streams, other host threads) race on the array and corrupt
+ *    each other's results; serialise them.
+ * Arguments and errors otherwise as mxa_decode_fwd. */
+MXA_API mxa_status_t mxa_decode_fwd_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                            const int32_t *block_table, const int32_t *cache_seqlens,
+                                            const mxa_decode_params_t *params, float scale, int causal,
+                                            int num_splits, void *out, float *lse, void *stream);
+
 /* Merge split results with the log-sum-exp identity (the reduce that
  * follows a KV-axis split, "Flash-Attention GQA 性能调优", section
  * "两个开关在 kernel 层面各做了什么"):
