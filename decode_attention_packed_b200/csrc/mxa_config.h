@@ -5,10 +5,13 @@
 
 namespace mxa {
 
-constexpr int kConsumerWarps = 4;                       // warps that do the math
-constexpr int kThreads = 32 * (kConsumerWarps + 1);     // + one producer (TMA) warp
+constexpr int kMathWarps = 4;                           // warps that run QK^T / softmax / PV
+constexpr int kProducerWarp = kMathWarps;               // TMA warp
+constexpr int kEpilogueWarp = kMathWarps + 1;           // cross-warp merge and output warp
+constexpr int kThreads = 32 * (kMathWarps + 2);
 constexpr int kRowsPerTile = 16;                        // packed query rows per tile (mma M)
 constexpr int kStages = 3;                              // depth of the K/V shared-memory ring
+constexpr int kJobs = 2;                                // epilogue hand-off slots
 constexpr int kSmemPerSm = 228 * 1024;                  // B200 shared memory per SM
 constexpr int kSmemReservedPerCta = 1024;               // driver-reserved shared memory per CTA
 constexpr int kMaxThreadsPerSm = 2048;
@@ -21,33 +24,40 @@ constexpr int block_tokens(int D) { return 8192 / D; }
 constexpr size_t stage_bytes(int D) { return (size_t)2 * block_tokens(D) * D * 2; }
 constexpr int q_row_pitch(int D) { return D * 2; }
 constexpr size_t q_tile_bytes(int D) { return (size_t)kRowsPerTile * q_row_pitch(D); }
-// fp32 scratch in which consumer warps 1..3 hand 8 rows of their output to warp 0
-constexpr size_t merge_bytes(int D) { return (size_t)(kConsumerWarps - 1) * 8 * D * 4; }
 
+// One unit of work for the math warps: a contiguous block range of one
+// (batch row, KV head, row tile) unit.
 struct SegmentDesc {
   int b, h, rt;          // batch row, KV head, row tile
   int blk_beg, blk_end;  // KV blocks [blk_beg, blk_end) of this unit
   int L;                 // valid keys of row b
-  int kind;              // 0 = whole unit (final output), 1 = head partial (slot 0),
-                         // 2 = tail partial (slot 1), -1 = end of work
-  int pad;
+  int kind;              // 0 = whole unit (final output), 1 = head piece (slot 0),
+                         // 2 = tail piece (slot 1), -1 = end of work
+  int c_first;           // first CTA holding a piece of the unit
+  int n_pieces;          // CTAs holding pieces of the unit
+  int pad[3];
 };
 
-constexpr size_t kBarrierBytes = 128;   // full[kStages], empty[kStages], qfull, qempty
-constexpr size_t kDescBytes = sizeof(SegmentDesc);
-constexpr size_t kMlBytes = (size_t)kConsumerWarps * kRowsPerTile * 2 * 4;
+// What the math warps hand to the epilogue warp at the end of a segment:
+// the segment, the ring stage that holds their partial outputs, and each
+// warp's running max and sum per packed row.
+struct JobSlot {
+  SegmentDesc seg;
+  int stage;
+  int pad[3];
+  float ml[kMathWarps][kRowsPerTile][2];
+};
+
+constexpr size_t kBarrierBytes = 128;   // full[S], empty[S], qfull, qempty, job_full[J], job_empty[J]
+constexpr int kNumBarriers = 2 * kStages + 2 + 2 * kJobs;
 
 // Offsets inside the dynamic shared memory (base aligned to 1024 bytes).
 constexpr size_t smem_ring_off() { return 0; }
 constexpr size_t smem_q_off(int D) { return smem_ring_off() + kStages * stage_bytes(D); }
-constexpr size_t smem_merge_off(int D) { return smem_q_off(D) + q_tile_bytes(D); }
-constexpr size_t smem_ml_off(int D) { return smem_merge_off(D) + merge_bytes(D); }
-constexpr size_t smem_desc_off(int D) { return smem_ml_off(D) + kMlBytes; }
-constexpr size_t smem_bar_off(int D) { return smem_desc_off(D) + kDescBytes; }
+constexpr size_t smem_desc_off(int D) { return smem_q_off(D) + q_tile_bytes(D); }
+constexpr size_t smem_jobs_off(int D) { return smem_desc_off(D) + sizeof(SegmentDesc); }
+constexpr size_t smem_bar_off(int D) { return smem_jobs_off(D) + kJobs * sizeof(JobSlot); }
 constexpr size_t smem_total(int D) { return smem_bar_off(D) + kBarrierBytes; }
-
-// Two CTAs per SM must fit: the ring, one Q tile, the merge scratch and the
-// barriers of each, plus the driver's per-CTA reservation.
 
 constexpr int ctas_per_sm(int D) {
   return (int)(kSmemPerSm / (smem_total(D) + kSmemReservedPerCta)) < (kMaxThreadsPerSm / kThreads)
@@ -55,21 +65,22 @@ constexpr int ctas_per_sm(int D) {
              : (kMaxThreadsPerSm / kThreads);
 }
 
-// Workspace: per-unit merge metadata, then two partial slots per CTA.
+// Workspace: per-unit arrival counters (epoch-tagged), then two partial
+// slots (head piece, tail piece) per CTA.
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-inline size_t ws_meta_bytes(long units) { return align256((size_t)units * 8); }
+inline size_t ws_count_bytes(long units) { return align256((size_t)units * 8); }
 inline size_t ws_lse_bytes(long grid) { return align256((size_t)grid * 2 * kRowsPerTile * 4); }
 inline size_t ws_o_bytes(long grid, int D) { return align256((size_t)grid * 2 * kRowsPerTile * D * 4); }
 inline size_t workspace_bytes(long units, long grid, int D) {
-  return ws_meta_bytes(units) + ws_lse_bytes(grid) + ws_o_bytes(grid, D);
+  return ws_count_bytes(units) + ws_lse_bytes(grid) + ws_o_bytes(grid, D);
 }
 
-}  // namespace mxa
-
-namespace mxa {
+static_assert(kNumBarriers * 8 <= (int)kBarrierBytes, "barrier area");
+static_assert(sizeof(SegmentDesc) % 16 == 0 && sizeof(JobSlot) % 16 == 0, "alignment");
 static_assert(2 * (smem_total(128) + kSmemReservedPerCta) <= (size_t)kSmemPerSm,
               "D = 128 layout must leave room for two CTAs per SM");
 static_assert(2 * (smem_total(64) + kSmemReservedPerCta) <= (size_t)kSmemPerSm,
               "D = 64 layout must leave room for two CTAs per SM");
-static_assert(smem_desc_off(128) % 16 == 0 && smem_bar_off(128) % 8 == 0, "alignment");
+static_assert((size_t)kMaxBalancedRows * 4 + 4 * 32 <= kStages * stage_bytes(64), "prologue scan fits the ring");
+
 }  // namespace mxa

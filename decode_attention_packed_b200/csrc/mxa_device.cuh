@@ -62,6 +62,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
+// Non-blocking test of the phase of `bar` with parity `parity`.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive_cnt(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
 // Wait for the phase of `bar` with parity `parity` to complete.  Returns
 // false (after recording `code` in *err_flag) if it has not completed within
 // kWaitLimitNs; the caller then stops its work instead of hanging the GPU.
@@ -78,17 +95,24 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
-// Warp-uniform bounded wait: lane 0 decides, every lane learns the outcome,
-// and on success every lane observes the completed phase itself (so that its
-// own later reads see what the phase published).  No lane can leave the warp
-// on a different path than the others.
+// Warp-uniform bounded wait: every lane polls the barrier itself and the
+// loop exits for all lanes together (on completion, seen by every lane, or
+// on timeout, seen by any lane).  Keeping the whole warp on one path
+// matters: a warp whose lanes wait on different paths (one lane polling,
+// the others parked at a shuffle) runs far slower afterwards.
 __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity, int *err_flag,
                                                   int code, int lane) {
-  bool ok = true;
-  if (lane == 0) ok = mbar_wait_bounded(bar, parity, err_flag, code);
-  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-  if (ok && lane != 0) mbar_wait_bounded(bar, parity, err_flag, code);  // completes at once
-  return ok;
+  bool mine = mbar_try_wait(bar, parity);
+  if (__all_sync(0xffffffffu, mine)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (!mine) mine = mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, mine)) return true;
+    if ((i & 63u) == 0 && __any_sync(0xffffffffu, globaltimer_ns() - t0 > kWaitLimitNs)) {
+      if (lane == 0) atomicOr(err_flag, code);
+      return false;
+    }
+  }
 }
 
 // 3-D tiled TMA load global -> shared, completing on `bar` (tx bytes).

@@ -1,10 +1,16 @@
 // Split-KV paged GQA decode attention for sm_100a.
 //
-// One kernel streams the KV cache: a producer warp gathers K/V pages through
-// the block table with TMA into a ring of shared-memory stages, and four
-// consumer warps run QK^T, the online softmax and PV on tensor cores
-// (m16n8k16, fp32 accumulation) over the packed query rows of one KV head.
-// A second, small kernel merges units whose KV axis was split across CTAs.
+// One kernel streams the KV cache.  Each CTA has three roles:
+//  - a producer warp gathers K/V pages through the block table with TMA
+//    into a ring of shared-memory stages, and brings each unit's packed Q
+//    rows in with bulk copies ahead of time;
+//  - four math warps run QK^T, the online softmax and PV on tensor cores
+//    (m16n8k16, fp32 accumulation) over the packed query rows of one KV
+//    head, each on its own slice of the keys of a stage;
+//  - an epilogue warp merges the math warps' partial results of a segment,
+//    writes the output (or a partial result when the unit is split across
+//    CTAs), and the CTA that completes a split unit merges its pieces with
+//    the log-sum-exp identity.
 //
 // Sources of the method:
 //  - "SmallQ FlashAttention (Vector)" README, 算法 (Algorithm): K-outer with
@@ -23,7 +29,9 @@
 //  - "MXFlashAttn 1.4.0" project page, 能力矩阵: paged KV cache, fp16/bf16,
 //    head_dim 64/128, grouped query heads.
 //  - "MixedQuantSparseFlashMlaMetadata 算子解析", 参数说明: the
-//    RightDownCausal mask for the draft tokens of a speculative step.
+//    RightDownCausal mask for the draft tokens of a speculative step; 源码级
+//    原理: a balanced division of the KV work over the cores, with a reduce
+//    for rows whose keys span several cores.
 #include "mxa_config.h"
 #include "mxa_device.cuh"
 #include "mxa_launch.h"
@@ -38,256 +46,378 @@ __device__ __forceinline__ int clamp_len(int L, int max_len) {
   return L < 0 ? 0 : (L > max_len ? max_len : L);
 }
 
+__device__ __forceinline__ uint32_t bar_addr(const uint8_t *smem, int D, int i) {
+  return smem_addr(smem + smem_bar_off(D)) + 8u * i;
+}
+// barrier indices
+constexpr int B_FULL(int s) { return s; }
+constexpr int B_EMPTY(int s) { return kStages + s; }
+constexpr int B_QFULL = 2 * kStages;
+constexpr int B_QEMPTY = 2 * kStages + 1;
+constexpr int B_JOBFULL(int j) { return 2 * kStages + 2 + j; }
+constexpr int B_JOBEMPTY(int j) { return 2 * kStages + 2 + kJobs + j; }
+
 // ---------------------------------------------------------------------------
-// Producer warp: walks this CTA's segments, loads each segment's packed Q
-// rows with bulk copies and every KV block of it with TMA tile loads.
+// Producer warp
 // ---------------------------------------------------------------------------
-template <int D>
-struct Walk {
-  // cursor over (row b, KV-head x row-tile hr, block blk) with `remaining`
-  // blocks left in this CTA's range
+
+// Cursor over this CTA's range of KV blocks: (row b, KV-head x row-tile hr,
+// block blk), `remaining` blocks left.
+struct Cursor {
   int b, hr, blk;
   long long remaining;
-  long long x;        // flattened index of the next block (balanced schedule)
+  long long x;        // flattened index of block blk (balanced schedule)
   long long per_cta;  // blocks per CTA range (balanced schedule)
-  int L, nb;
+  int L, nb;          // length and blocks of row b
+  int L_next;         // prefetched length of row b + 1
 };
 
 template <int D>
-__device__ __forceinline__ void walk_load_row(Walk<D> &w, const DecodeArgs &a) {
-  w.L = clamp_len(a.seqlens[w.b], a.max_seqlen_k);
-  w.nb = (w.L + block_tokens(D) - 1) / block_tokens(D);
+__device__ __forceinline__ void cursor_enter_row(Cursor &c, const DecodeArgs &a, int L) {
+  constexpr int T = block_tokens(D);
+  c.L = L;
+  c.nb = (L + T - 1) / T;
+  c.L_next = c.b + 1 < a.B ? a.seqlens[c.b + 1] : 0;  // consumed a segment later
 }
 
-// Skip rows without blocks (L_b = 0); they hold no work for the walk.
+// The segment at the cursor (a contiguous block range of one unit); the
+// cursor moves past it.
 template <int D>
-__device__ __forceinline__ void walk_skip_empty(Walk<D> &w, const DecodeArgs &a) {
-  while (w.remaining > 0 && w.nb == 0 && w.b + 1 < a.B) {
-    ++w.b;
-    w.hr = 0;
-    w.blk = 0;
-    walk_load_row(w, a);
+__device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
+  const int HR = a.Hkv * a.RT;
+  SegmentDesc s;
+  const long long left = c.nb - c.blk;
+  const int len = (int)(left < c.remaining ? left : c.remaining);
+  s.b = c.b;
+  s.h = c.hr / a.RT;
+  s.rt = c.hr % a.RT;
+  s.blk_beg = c.blk;
+  s.blk_end = c.blk + len;
+  s.L = c.L;
+  s.kind = (s.blk_beg == 0 && s.blk_end == c.nb) ? 0 : (s.blk_beg > 0 ? 1 : 2);
+  if (a.schedule == MXA_SCHED_BALANCED) {
+    const long long xs = c.x - c.blk;  // flattened index of the unit's first block
+    s.c_first = (int)(xs / c.per_cta);
+    s.n_pieces = (int)((xs + c.nb - 1) / c.per_cta) - s.c_first + 1;
+  } else {
+    const int unit = (c.b * a.Hkv + s.h) * a.RT + s.rt;
+    s.c_first = unit * a.splits;
+    s.n_pieces = (c.nb + a.chunk_blocks - 1) / a.chunk_blocks;
   }
+  s.pad[0] = s.pad[1] = s.pad[2] = 0;
+
+  c.remaining -= len;
+  c.x += len;
+  c.blk += len;
+  if (c.blk == c.nb) {
+    c.blk = 0;
+    if (++c.hr == HR) {
+      c.hr = 0;
+      if (c.remaining > 0 && c.b + 1 < a.B) {
+        ++c.b;
+        cursor_enter_row<D>(c, a, clamp_len(c.L_next, a.max_seqlen_k));
+        while (c.nb == 0 && c.b + 1 < a.B) {  // rows without keys hold no blocks
+          ++c.b;
+          cursor_enter_row<D>(c, a, clamp_len(a.seqlens[c.b], a.max_seqlen_k));
+        }
+      } else {
+        c.remaining = 0;
+      }
+    }
+  }
+  return s;
+}
+
+// This CTA's range of the flattened block space.  BALANCED: the blocks of
+// all units laid end to end (row-major over (b, KV head, row tile)) and cut
+// into gridDim.x equal ranges; the prefix sum over rows is built in the
+// (still unused) ring by this warp alone.  UNIFORM: block range
+// [si * chunk, (si + 1) * chunk) of unit blockIdx.x / splits.
+template <int D>
+__device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane) {
+  constexpr int T = block_tokens(D);
+  const int HR = a.Hkv * a.RT;
+  Cursor c;
+  c.hr = 0;
+  c.blk = 0;
+  c.remaining = 0;
+  c.x = 0;
+  c.per_cta = 1;
+  c.L = c.nb = c.L_next = 0;
+  if (a.schedule == MXA_SCHED_UNIFORM) {
+    const int u = blockIdx.x / a.splits, si = blockIdx.x % a.splits;
+    c.b = u / HR;
+    c.hr = u % HR;
+    c.L = clamp_len(a.seqlens[c.b], a.max_seqlen_k);
+    c.nb = (c.L + T - 1) / T;
+    const int beg = si * a.chunk_blocks, end = min(beg + a.chunk_blocks, c.nb);
+    c.blk = beg;
+    c.remaining = end > beg ? end - beg : 0;
+    c.L_next = 0;
+    return c;
+  }
+  int *scan = reinterpret_cast<int *>(smem + smem_ring_off());
+  const int chunk = (a.B + 31) / 32;
+  const int lo = min(lane * chunk, a.B), hi = min(lo + chunk, a.B);
+  int sum = 0;
+  for (int i = lo; i < hi; ++i) {
+    const int nb = (clamp_len(a.seqlens[i], a.max_seqlen_k) + T - 1) / T;
+    scan[i] = nb;
+    sum += nb;
+  }
+  __syncwarp();
+  int incl = sum;  // inclusive warp scan of the lane sums
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  int run = incl - sum;
+  for (int i = lo; i < hi; ++i) {
+    run += scan[i];
+    scan[i] = run;  // inclusive prefix of blocks per row
+  }
+  __syncwarp();
+  const long long NB = (long long)HR * total;
+  c.per_cta = NB == 0 ? 1 : (NB + gridDim.x - 1) / gridDim.x;
+  const long long x0 = (long long)blockIdx.x * c.per_cta;
+  c.b = 0;
+  if (x0 < NB) {
+    int lo_b = 0, hi_b = a.B - 1;  // first row whose blocks end past x0
+    while (lo_b < hi_b) {
+      const int mid = (lo_b + hi_b) >> 1;
+      if ((long long)HR * scan[mid] > x0) hi_b = mid; else lo_b = mid + 1;
+    }
+    const long long pre = lo_b > 0 ? scan[lo_b - 1] : 0;
+    const long long nb = scan[lo_b] - pre;
+    const long long off = x0 - (long long)HR * pre;
+    c.b = lo_b;
+    c.hr = (int)(off / nb);
+    c.blk = (int)(off % nb);
+    c.remaining = c.per_cta < NB - x0 ? c.per_cta : NB - x0;
+    c.x = x0;
+    c.nb = (int)nb;  // from the scan: the length itself is first needed later
+    c.L = clamp_len(a.seqlens[c.b], a.max_seqlen_k);
+    c.L_next = c.b + 1 < a.B ? a.seqlens[c.b + 1] : 0;
+  }
+  __syncwarp();
+  fence_proxy_async_smem();  // these generic writes precede the TMA writes to the ring
+  return c;
+}
+
+// Block-table window of the producer warp: lane i holds the page ids of
+// logical pages base + i (wa) and base + 32 + i (wb) of row b.
+struct Window {
+  int base, wa, wb;
+};
+
+__device__ __forceinline__ int bt_entry(const DecodeArgs &a, int b, int p, int npages) {
+  return p < npages ? a.block_table[(size_t)b * a.mpps + p] : 0;
 }
 
 template <int D, bool kBf16>
-__device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, Walk<D> w, uint8_t *smem,
-                              int lane) {
+__device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *smem, int lane) {
   constexpr int T = block_tokens(D);
   constexpr int CH = D / 64;
   constexpr uint32_t KV_BYTES = (uint32_t)T * D * 2;
   const uint32_t ring = smem_addr(smem + smem_ring_off());
   const uint32_t qtile = smem_addr(smem + smem_q_off(D));
-  const uint32_t bar0 = smem_addr(smem + smem_bar_off(D));
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-  const uint32_t qfull = bar0 + 8u * (2 * kStages);
-  const uint32_t qempty = bar0 + 8u * (2 * kStages + 1);
+  const uint32_t qfull = bar_addr(smem, D, B_QFULL), qempty = bar_addr(smem, D, B_QEMPTY);
   SegmentDesc *desc = reinterpret_cast<SegmentDesc *>(smem + smem_desc_off(D));
-
-  const int HR = a.Hkv * a.RT;
   const int bt = a.box_tokens;
+  const int ps = a.page_size;
   const uint16_t *q = reinterpret_cast<const uint16_t *>(a.q);
 
   if (lane == 0) {
     prefetch_tmap(&tm.k);
     prefetch_tmap(&tm.v);
   }
+  Cursor cur = cursor_start<D>(a, smem, lane);
 
-  int it = 0;     // KV stages issued
-  int seg_k = 0;  // segments issued
-  int win_b = -1, win_base = 0, win_val = 0;  // block-table window: lane i holds entry win_base + i
-  bool ok = true;
-
-  while (ok && w.remaining > 0 && w.nb > 0) {
-    const int seg_len = (int)((long long)(w.nb - w.blk) < w.remaining ? (w.nb - w.blk) : w.remaining);
-    const int blk_beg = w.blk, blk_end = w.blk + seg_len;
-    const int h = w.hr / a.RT, rt = w.hr % a.RT;
-    const int kind = (blk_beg == 0 && blk_end == w.nb) ? 0 : (blk_beg > 0 ? 1 : 2);
-    const int rows = min(kRowsPerTile, a.M - rt * kRowsPerTile);
-    const int unit = (w.b * a.Hkv + h) * a.RT + rt;
-
-    // first block of a unit: record which CTAs hold its pieces
-    if (blk_beg == 0 && lane == 0 && a.meta != nullptr) {
-      int c_last;
-      if (a.schedule == MXA_SCHED_BALANCED) {
-        c_last = (int)((w.x + w.nb - 1) / w.per_cta);
-      } else {
-        c_last = (int)blockIdx.x + (w.nb + a.chunk_blocks - 1) / a.chunk_blocks - 1;
-      }
-      a.meta[unit] = make_int2((int)blockIdx.x, c_last);
-    }
-
-    // ---- Q tile of this unit (packed rows m = t * G + g) ----
-    if (!warp_wait_bounded(qempty, (seg_k & 1) ^ 1, &g_mxa_err, kErrWaitQ, lane)) { ok = false; break; }
+  // Publish a segment to the math warps: its descriptor and its Q tile.
+  auto issue_q = [&](const SegmentDesc &s) {
+    const int rows = min(kRowsPerTile, a.M - s.rt * kRowsPerTile);
     if (lane == 0) {
-      SegmentDesc d;
-      d.b = w.b; d.h = h; d.rt = rt; d.blk_beg = blk_beg; d.blk_end = blk_end;
-      d.L = w.L; d.kind = kind; d.pad = 0;
-      *desc = d;
+      *desc = s;
       mbar_arrive_expect_tx(qfull, (uint32_t)rows * D * 2);
     }
     __syncwarp();
     if (lane < rows) {
-      const int m = rt * kRowsPerTile + lane;
+      const int m = s.rt * kRowsPerTile + lane;
       const int t = m / a.G, g = m % a.G;
-      const uint16_t *src = q + ((size_t)(w.b * a.q_len + t) * a.Hq + (size_t)h * a.G + g) * D;
+      const uint16_t *src = q + ((size_t)(s.b * a.q_len + t) * a.Hq + (size_t)s.h * a.G + g) * D;
       bulk_load(qtile + (uint32_t)lane * q_row_pitch(D), src, D * 2, qfull);
     }
-    ++seg_k;
+  };
+  // Entries past a row's last page are never used for a load; bounding by
+  // the table's row width lets the window be read before L_b is known.
+  auto load_window = [&](const SegmentDesc &s, Window &w) {
+    w.base = 0;
+    w.wa = w.wb = 0;
+    if (a.contiguous) return;
+    w.base = (s.blk_beg * T) / ps;
+    w.wa = bt_entry(a, s.b, w.base + lane, a.mpps);
+    w.wb = bt_entry(a, s.b, w.base + 32 + lane, a.mpps);
+  };
 
-    // ---- KV blocks ----
-    const int npages_b = a.contiguous ? 1 : (w.L + a.page_size - 1) / a.page_size;
-    for (int blk = blk_beg; blk < blk_end; ++blk) {
-      const int s = it % kStages;
-      const int k = it / kStages;
-      const int tok0 = blk * T;
-      const int valid = min(T, w.L - tok0);
-      const int nbox = (valid + bt - 1) / bt;
-
-      int page_src_lane = 0;
-      if (!a.contiguous) {
-        const int first = tok0 / a.page_size;
-        const int last = (tok0 + (nbox - 1) * bt) / a.page_size;
-        if (win_b != w.b || first < win_base || last >= win_base + 32) {
-          win_b = w.b;
-          win_base = first;
-          const int e = win_base + lane;
-          win_val = e < npages_b ? a.block_table[(size_t)w.b * a.mpps + e] : 0;
-        }
-      }
-      const int n_ops = nbox * CH * 2;
-      const int box = lane / (CH * 2);
-      const int ch = (lane / 2) % CH;
-      const int kv = lane & 1;
-      const int tok = tok0 + box * bt;
-      if (!a.contiguous) {
-        int idx = tok / a.page_size - win_base;
-        page_src_lane = idx < 0 ? 0 : (idx > 31 ? 31 : idx);
-      }
-      const int page = __shfl_sync(0xffffffffu, win_val, page_src_lane);
-
-      if (!warp_wait_bounded(empty_bar(s), (k & 1) ^ 1, &g_mxa_err, kErrWaitEmpty, lane)) { ok = false; break; }
-      if (lane == 0) mbar_arrive_expect_tx(full_bar(s), (uint32_t)nbox * bt * D * 2 * 2);
-      __syncwarp();
-      if (lane < n_ops) {
-        const int row = a.contiguous ? w.b * a.page_size + tok
-                                     : page * a.page_size + tok % a.page_size;
-        const uint32_t dst = ring + (uint32_t)s * (2 * KV_BYTES) + (uint32_t)kv * KV_BYTES +
-                             (uint32_t)ch * (T * 128) + (uint32_t)(box * bt) * 128;
-        tma_load_3d(dst, kv ? (const void *)&tm.v : (const void *)&tm.k, ch * 64, h, row, full_bar(s));
-      }
-      ++it;
+  int it = 0;     // KV stages issued
+  int seg_k = 0;  // segments published
+  bool ok = true;
+  if (cur.remaining > 0 && cur.nb > 0) {
+    SegmentDesc seg = cursor_take<D>(cur, a);
+    Window win;
+    load_window(seg, win);
+    if (!warp_wait_bounded(qempty, 1, &g_mxa_err, kErrWaitQ, lane)) ok = false;  // first use: free
+    if (ok) {
+      issue_q(seg);
+      ++seg_k;
     }
-    if (!ok) break;
-
-    // advance the cursor past this segment
-    w.remaining -= seg_len;
-    w.x += seg_len;
-    w.blk = blk_end;
-    if (w.blk == w.nb) {
-      w.blk = 0;
-      if (++w.hr == HR) {
-        w.hr = 0;
-        if (w.remaining > 0 && w.b + 1 < a.B) {
-          ++w.b;
-          walk_load_row(w, a);
-          walk_skip_empty(w, a);
-        } else {
-          w.remaining = 0;
+    while (ok) {
+      const bool have_next = cur.remaining > 0 && cur.nb > 0;
+      SegmentDesc nseg;
+      Window nwin;
+      bool q_next = false;
+      if (have_next) {
+        nseg = cursor_take<D>(cur, a);
+        load_window(nseg, nwin);  // its latency hides behind this segment's stages
+      }
+      for (int blk = seg.blk_beg; blk < seg.blk_end; ++blk) {
+        const int s = it % kStages;
+        const int k = it / kStages;
+        const int tok0 = blk * T;
+        const int valid = min(T, seg.L - tok0);
+        const int nbox = (valid + bt - 1) / bt;
+        const int n_ops = nbox * CH * 2;
+        const int box = lane / (CH * 2);
+        const int ch = (lane / 2) % CH;
+        const int kv = lane & 1;
+        const int tok = tok0 + box * bt;
+        int page = 0;
+        if (!a.contiguous) {
+          if (tok0 / ps - win.base >= 32) {  // slide the window by 32 pages
+            win.base += 32;
+            win.wa = win.wb;
+            win.wb = bt_entry(a, seg.b, win.base + 32 + lane, a.mpps);
+          }
+          const int idx = tok / ps - win.base;
+          const int src = idx & 31;
+          const int va = __shfl_sync(0xffffffffu, win.wa, src);
+          const int vb = __shfl_sync(0xffffffffu, win.wb, src);
+          page = idx < 32 ? va : vb;
+        }
+        if (!warp_wait_bounded(bar_addr(smem, D, B_EMPTY(s)), (k & 1) ^ 1, &g_mxa_err, kErrWaitEmpty,
+                               lane)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(bar_addr(smem, D, B_FULL(s)), (uint32_t)nbox * bt * D * 2 * 2);
+        __syncwarp();
+        if (lane < n_ops) {
+          const int row = a.contiguous ? seg.b * ps + tok : page * ps + tok % ps;
+          const uint32_t dst = ring + (uint32_t)s * (2 * KV_BYTES) + (uint32_t)kv * KV_BYTES +
+                               (uint32_t)ch * (T * 128) + (uint32_t)(box * bt) * 128;
+          tma_load_3d(dst, kv ? (const void *)&tm.v : (const void *)&tm.k, ch * 64, seg.h, row,
+                      bar_addr(smem, D, B_FULL(s)));
+        }
+        ++it;
+        // publish the next segment as soon as the math warps hold this one's Q
+        if (have_next && !q_next) {
+          bool free_slot = false;
+          if (lane == 0) free_slot = mbar_test_wait(qempty, (seg_k & 1) ^ 1);
+          if (__shfl_sync(0xffffffffu, free_slot ? 1 : 0, 0)) {
+            issue_q(nseg);
+            ++seg_k;
+            q_next = true;
+          }
         }
       }
+      if (!ok || !have_next) break;
+      if (!q_next) {
+        if (!warp_wait_bounded(qempty, (seg_k & 1) ^ 1, &g_mxa_err, kErrWaitQ, lane)) {
+          ok = false;
+          break;
+        }
+        issue_q(nseg);
+        ++seg_k;
+      }
+      seg = nseg;
+      win = nwin;
     }
   }
 
-  grid_launch_dependents();
-
-  if (ok) {
-    // end-of-work marker for the consumers
-    if (warp_wait_bounded(qempty, (seg_k & 1) ^ 1, &g_mxa_err, kErrWaitQ, lane)) {
-      if (lane == 0) {
-        SegmentDesc d{};
-        d.kind = -1;
-        *desc = d;
-        mbar_arrive(qfull);
-      }
-      return;
+  if (ok && warp_wait_bounded(qempty, (seg_k & 1) ^ 1, &g_mxa_err, kErrWaitQ, lane)) {
+    if (lane == 0) {  // end-of-work marker for the math warps
+      SegmentDesc d{};
+      d.kind = -1;
+      *desc = d;
+      mbar_arrive(qfull);
     }
+    return;
   }
-  // Failure path: do not leave the CTA while copies this warp issued may
-  // still be writing shared memory.  Wait (bounded) for the last stages.
+  // Failure path: do not leave while copies this warp issued may still be
+  // writing shared memory.  Wait (bounded) for the last stages and Q tile.
   const int n_inflight = it < kStages ? it : kStages;
-  for (int j = it - n_inflight; j < it; ++j) {
-    mbar_wait_bounded(full_bar(j % kStages), (j / kStages) & 1, &g_mxa_err, kErrDrain);
-  }
+  for (int j = it - n_inflight; j < it; ++j)
+    mbar_wait_bounded(bar_addr(smem, D, B_FULL(j % kStages)), (j / kStages) & 1, &g_mxa_err, kErrDrain);
   if (seg_k > 0) mbar_wait_bounded(qfull, (seg_k - 1) & 1, &g_mxa_err, kErrDrain);
 }
 
 // ---------------------------------------------------------------------------
-// Consumer warps
+// Math warps
 // ---------------------------------------------------------------------------
 
-// Output of a unit whose row sees no key at all (L_b = 0): O = 0, LSE = -inf.
+// Address of fp32 element (row, col) of math warp `warp`'s partial output
+// inside its own key slice of ring stage `sbase` (the segment's last stage,
+// which the warp has finished reading).  Rows of D floats; the 16-byte
+// chunks of a row are XOR-swizzled by the row index against bank conflicts.
 template <int D>
-__device__ void write_empty_unit(const DecodeArgs &a, int unit, int tid) {
-  const int rt = unit % a.RT, hr = unit / a.RT, h = hr % a.Hkv, b = hr / a.Hkv;
-  const int rows = min(kRowsPerTile, a.M - rt * kRowsPerTile);
-  uint16_t *out = reinterpret_cast<uint16_t *>(a.out);
-  for (int i = tid; i < rows * D; i += kConsumerWarps * 32) {
-    const int rr = i / D, d = i % D;
-    const int m = rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G;
-    out[((size_t)(b * a.q_len + t) * a.Hq + (size_t)h * a.G + g) * D + d] = 0;  // +0 in fp16 and bf16
-  }
-  if (a.lse != nullptr) {
-    for (int rr = tid; rr < rows; rr += kConsumerWarps * 32) {
-      const int m = rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G;
-      a.lse[((size_t)b * a.Hq + (size_t)h * a.G + g) * a.q_len + t] = -INFINITY;
-    }
-  }
-  if (tid == 0 && a.meta != nullptr) a.meta[unit] = make_int2((int)blockIdx.x, (int)blockIdx.x);
+__device__ __forceinline__ uint32_t handoff_addr(uint32_t sbase, int warp, int row, int col) {
+  constexpr int T = block_tokens(D);
+  constexpr int TW = T / kMathWarps;
+  constexpr int CH = D / 64;
+  constexpr uint32_t KV_BYTES = (uint32_t)T * D * 2;
+  const uint32_t ro = (uint32_t)row * D * 4;
+  const uint32_t piece = ro / (TW * 128), within = ro % (TW * 128);
+  const uint32_t region = sbase + (piece >= (uint32_t)CH ? KV_BYTES : 0u) + (piece % CH) * (T * 128) +
+                          (uint32_t)warp * TW * 128;
+  const uint32_t chunk = (uint32_t)(col >> 2) ^ (uint32_t)(row & 7);
+  return region + within + (chunk << 4) + ((uint32_t)(col & 3) << 2);
 }
 
 template <int D, bool kBf16>
-__device__ void consumer_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lane) {
+__device__ void math_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lane) {
   constexpr int T = block_tokens(D);
-  constexpr int TW = T / kConsumerWarps;  // tokens of one warp per stage
-  constexpr int NT = TW / 8;              // score n-tiles of one warp per stage
-  constexpr int KS = D / 16;              // k-steps of Q K^T
-  constexpr int DN = D / 8;               // n-tiles of the output
+  constexpr int TW = T / kMathWarps;  // keys of one warp per stage
+  constexpr int NT = TW / 8;          // score n-tiles of one warp per stage
+  constexpr int KS = D / 16;          // k-steps of Q K^T
+  constexpr int DN = D / 8;           // n-tiles of the output
   constexpr uint32_t KV_BYTES = (uint32_t)T * D * 2;
   constexpr float NEG_INF = -INFINITY;
 
   const uint32_t ring = smem_addr(smem + smem_ring_off());
   const uint32_t qtile = smem_addr(smem + smem_q_off(D));
-  const uint32_t bar0 = smem_addr(smem + smem_bar_off(D));
-  const uint32_t qfull = bar0 + 8u * (2 * kStages);
-  const uint32_t qempty = bar0 + 8u * (2 * kStages + 1);
-  const uint32_t epbar = bar0 + 8u * (2 * kStages + 2);  // epilogue sync of the consumer warps
+  const uint32_t qfull = bar_addr(smem, D, B_QFULL), qempty = bar_addr(smem, D, B_QEMPTY);
   const volatile int *desc = reinterpret_cast<const volatile int *>(smem + smem_desc_off(D));
-  float *ml = reinterpret_cast<float *>(smem + smem_ml_off(D));
-  float *merge = reinterpret_cast<float *>(smem + smem_merge_off(D));
+  JobSlot *jobs = reinterpret_cast<JobSlot *>(smem + smem_jobs_off(D));
 
   const int r = lane >> 2, c = lane & 3;
   const float sl2 = a.scale_log2;
 
-  // Consumer-group barrier with a bounded wait (a warp that gave up on a
-  // wait returns; the others then give up here instead of hanging).
-  int ep_k = 0;
-  auto ep_sync = [&]() -> bool {
-    __syncwarp();
-    if (lane == 0) mbar_arrive(epbar);
-    const bool ok = warp_wait_bounded(epbar, ep_k & 1, &g_mxa_err, kErrWaitFull, lane);
-    ++ep_k;
-    return ok;
-  };
-
   int it = 0, seg_k = 0;
   for (;;) {
     if (!warp_wait_bounded(qfull, seg_k & 1, &g_mxa_err, kErrWaitQ, lane)) return;
-    const int kind = desc[6];
-    if (kind < 0) return;
     const int b = desc[0], h = desc[1], rt = desc[2], blk_beg = desc[3], blk_end = desc[4];
-    const int L = desc[5];
+    const int L = desc[5], kind = desc[6], c_first = desc[7], n_pieces = desc[8];
+    const int j = seg_k % kJobs, jk = seg_k / kJobs;
+    if (kind < 0) {  // end of work: pass the marker on to the epilogue warp
+      if (!warp_wait_bounded(bar_addr(smem, D, B_JOBEMPTY(j)), (jk & 1) ^ 1, &g_mxa_err, kErrWaitQ, lane))
+        return;
+      if (warp == 0 && lane == 0) jobs[j].seg.kind = -1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_addr(smem, D, B_JOBFULL(j)));
+      return;
+    }
     const int rows = min(kRowsPerTile, a.M - rt * kRowsPerTile);
 
     // Q tile -> A fragments, resident in registers for the whole segment
@@ -319,10 +449,11 @@ __device__ void consumer_warps(const DecodeArgs &a, uint8_t *smem, int warp, int
 #pragma unroll
     for (int dn = 0; dn < DN; ++dn) o[dn][0] = o[dn][1] = o[dn][2] = o[dn][3] = 0.f;
 
+    int s_last = 0;
     for (int blk = blk_beg; blk < blk_end; ++blk) {
       const int s = it % kStages;
       const int k = it / kStages;
-      if (!warp_wait_bounded(bar0 + 8u * s, k & 1, &g_mxa_err, kErrWaitFull, lane)) return;
+      if (!warp_wait_bounded(bar_addr(smem, D, B_FULL(s)), k & 1, &g_mxa_err, kErrWaitFull, lane)) return;
       const uint32_t kbase = ring + (uint32_t)s * (2 * KV_BYTES);
       const uint32_t vbase = kbase + KV_BYTES;
       const int j0 = blk * T + warp * TW;  // first key of this warp's slice
@@ -371,9 +502,9 @@ __device__ void consumer_warps(const DecodeArgs &a, uint8_t *smem, int warp, int
         for (int e = 0; e < 2; ++e) {
           float x0 = sc[nt][e] * sl2, x1 = sc[nt][2 + e] * sl2;
           if (need_mask) {
-            const int j = j0 + nt * 8 + 2 * c + e;
-            x0 = j < lim0 ? x0 : NEG_INF;
-            x1 = j < lim1 ? x1 : NEG_INF;
+            const int jj = j0 + nt * 8 + 2 * c + e;
+            x0 = jj < lim0 ? x0 : NEG_INF;
+            x1 = jj < lim1 ? x1 : NEG_INF;
           }
           sc[nt][e] = x0;
           sc[nt][2 + e] = x1;
@@ -438,276 +569,323 @@ __device__ void consumer_warps(const DecodeArgs &a, uint8_t *smem, int warp, int
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar0 + 8u * (kStages + s));
+      if (blk + 1 < blk_end) {
+        if (lane == 0) mbar_arrive(bar_addr(smem, D, B_EMPTY(s)));
+      } else {
+        s_last = s;  // kept for the hand-off; the epilogue warp releases it
+      }
       ++it;
     }
 
-    // ---- epilogue: merge the four warps' (m, l, O) of this segment ----
+    // ---- hand-off: (m, l) per row and the unnormalised O of this warp ----
+    if (!warp_wait_bounded(bar_addr(smem, D, B_JOBEMPTY(j)), (jk & 1) ^ 1, &g_mxa_err, kErrWaitQ, lane))
+      return;
     l_0 += __shfl_xor_sync(0xffffffffu, l_0, 1);
     l_0 += __shfl_xor_sync(0xffffffffu, l_0, 2);
     l_1 += __shfl_xor_sync(0xffffffffu, l_1, 1);
     l_1 += __shfl_xor_sync(0xffffffffu, l_1, 2);
     if (c == 0) {
-      ml[(warp * 16 + r) * 2] = m_0;
-      ml[(warp * 16 + r) * 2 + 1] = l_0;
-      ml[(warp * 16 + r + 8) * 2] = m_1;
-      ml[(warp * 16 + r + 8) * 2 + 1] = l_1;
+      jobs[j].ml[warp][r][0] = m_0;
+      jobs[j].ml[warp][r][1] = l_0;
+      jobs[j].ml[warp][r + 8][0] = m_1;
+      jobs[j].ml[warp][r + 8][1] = l_1;
     }
-    if (!ep_sync()) return;
-    float Mx0 = NEG_INF, Mx1 = NEG_INF;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      Mx0 = fmaxf(Mx0, ml[(w * 16 + r) * 2]);
-      Mx1 = fmaxf(Mx1, ml[(w * 16 + r + 8) * 2]);
-    }
-    float Lx0 = 0.f, Lx1 = 0.f;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      const float mw0 = ml[(w * 16 + r) * 2], mw1 = ml[(w * 16 + r + 8) * 2];
-      if (mw0 != NEG_INF) Lx0 += ex2(mw0 - Mx0) * ml[(w * 16 + r) * 2 + 1];
-      if (mw1 != NEG_INF) Lx1 += ex2(mw1 - Mx1) * ml[(w * 16 + r + 8) * 2 + 1];
-    }
-    const float f0 = (m_0 != NEG_INF && Lx0 > 0.f) ? ex2(m_0 - Mx0) / Lx0 : 0.f;
-    const float f1 = (m_1 != NEG_INF && Lx1 > 0.f) ? ex2(m_1 - Mx1) / Lx1 : 0.f;
-    const float lse0 = Lx0 > 0.f ? (Mx0 + log2f(Lx0)) * kLn2 : NEG_INF;
-    const float lse1 = Lx1 > 0.f ? (Mx1 + log2f(Lx1)) * kLn2 : NEG_INF;
+    const uint32_t sbase = ring + (uint32_t)s_last * (2 * KV_BYTES);
 #pragma unroll
     for (int dn = 0; dn < DN; ++dn) {
-      o[dn][0] *= f0;
-      o[dn][1] *= f0;
-      o[dn][2] *= f1;
-      o[dn][3] *= f1;
+      const int col = dn * 8 + 2 * c;
+      if (r < rows)
+        asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(handoff_addr<D>(sbase, warp, r, col)),
+                     "f"(o[dn][0]), "f"(o[dn][1]) : "memory");
+      if (r + 8 < rows)
+        asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(handoff_addr<D>(sbase, warp, r + 8, col)),
+                     "f"(o[dn][2]), "f"(o[dn][3]) : "memory");
     }
-    const int npass = rows > 8 ? 2 : 1;
-    const int slot = kind - 1;  // partial slot (kind 1 -> 0, kind 2 -> 1)
-    for (int hf = 0; hf < npass; ++hf) {
-      if (hf && !ep_sync()) return;  // warp 0 has read the first half
-      if (warp > 0) {
+    if (warp == 0 && lane == 0) {
+      SegmentDesc sd;
+      sd.b = b; sd.h = h; sd.rt = rt; sd.blk_beg = blk_beg; sd.blk_end = blk_end; sd.L = L;
+      sd.kind = kind; sd.c_first = c_first; sd.n_pieces = n_pieces;
+      sd.pad[0] = sd.pad[1] = sd.pad[2] = 0;
+      jobs[j].seg = sd;
+      jobs[j].stage = s_last;
+    }
+    fence_proxy_async_smem();  // the stage returns to TMA after the epilogue warp has read it
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_addr(smem, D, B_JOBFULL(j)));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Epilogue warp
+// ---------------------------------------------------------------------------
+
+// D / 32 consecutive output values of one row -> out[b, t, hq, col..]
+template <int D, bool kBf16>
+__device__ __forceinline__ void store_out_vec(const DecodeArgs &a, int b, int t, int hq, int col,
+                                              const float *v) {
+  uint16_t *dst = reinterpret_cast<uint16_t *>(a.out) + ((size_t)(b * a.q_len + t) * a.Hq + hq) * D + col;
+  if constexpr (D / 32 == 4) {
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(pack2<kBf16>(v[0], v[1]), pack2<kBf16>(v[2], v[3]));
+  } else {
+    *reinterpret_cast<uint32_t *>(dst) = pack2<kBf16>(v[0], v[1]);
+  }
+}
+
+// Output of a unit whose row sees no key at all (L_b = 0): O = 0, LSE = -inf.
+template <int D>
+__device__ void write_empty_unit(const DecodeArgs &a, int unit, int lane) {
+  const int rt = unit % a.RT, hr = unit / a.RT, h = hr % a.Hkv, b = hr / a.Hkv;
+  const int rows = min(kRowsPerTile, a.M - rt * kRowsPerTile);
+  uint16_t *out = reinterpret_cast<uint16_t *>(a.out);
+  for (int i = lane; i < rows * D; i += 32) {
+    const int rr = i / D, d = i % D;
+    const int m = rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G;
+    out[((size_t)(b * a.q_len + t) * a.Hq + (size_t)h * a.G + g) * D + d] = 0;  // +0 in fp16 and bf16
+  }
+  if (a.lse != nullptr) {
+    for (int rr = lane; rr < rows; rr += 32) {
+      const int m = rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G;
+      a.lse[((size_t)b * a.Hq + (size_t)h * a.G + g) * a.q_len + t] = -INFINITY;
+    }
+  }
+  __syncwarp();
+}
+
+// Count this piece of a split unit; true (in every lane) for the piece that
+// completes it.  The counter carries the call's epoch in its high half, so a
+// count left by an earlier (failed) call is not mistaken for this call's.
+// The retry loop runs on all lanes; only lane 0 touches memory.
+__device__ __forceinline__ bool arrive_and_check_last(const DecodeArgs &a, int unit, int n, int lane) {
+  unsigned long long *cnt = a.counters + unit;
+  const unsigned long long ep = a.epoch;
+  unsigned long long cur = 0;
+  if (lane == 0) cur = atomicAdd(cnt, 0ull);
+  cur = __shfl_sync(0xffffffffu, cur, 0);
+  for (;;) {
+    const unsigned long long want = (cur >> 32) == ep ? cur + 1ull : ((ep << 32) | 1ull);
+    unsigned long long prev = 0;
+    if (lane == 0) prev = atomicCAS(cnt, cur, want);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (prev == cur) return (int)(want & 0xffffffffull) == n;
+    cur = prev;
+  }
+}
+
+// Merge the n pieces of a split unit with the log-sum-exp identity:
+// LSE = ln sum_i exp(lse_i), O = sum_i exp(lse_i - LSE) O_i.  The pieces are
+// the tail slot of the first CTA and the head slots of the following ones.
+// Lane r < rows owns the statistics of packed row r; every lane owns D / 32
+// output columns of every row.  Loads of one round are independent, so a
+// merge costs a few memory round trips whatever the number of rows.
+template <int D, bool kBf16>
+__device__ void merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int rows, int unit, int lane) {
+  constexpr int VEC = D / 32;
+  const int n = sg.n_pieces, cf = sg.c_first;
+  auto slot_of = [&](int i) -> size_t { return i == 0 ? (size_t)cf * 2 + 1 : (size_t)(cf + i) * 2; };
+  const int col = lane * VEC;
+  // statistics of row `lane`, one pass with a running maximum (loads of a
+  // batch of 8 pieces are issued together)
+  float mx = -INFINITY, sum = 0.f;
+  {
+    const bool mine = lane < rows;  // all lanes run the loop; only rows' lanes load
+    for (int i0 = 0; i0 < n; i0 += 8) {
+      float l[8];
 #pragma unroll
-        for (int dn = 0; dn < DN; ++dn)
-          *reinterpret_cast<float2 *>(&merge[((warp - 1) * 8 + r) * D + dn * 8 + 2 * c]) =
-              make_float2(o[dn][2 * hf], o[dn][2 * hf + 1]);
+      for (int q = 0; q < 8; ++q)
+        l[q] = (mine && i0 + q < n) ? __ldcg(a.lse_part + slot_of(i0 + q) * kRowsPerTile + lane) : -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (l[q] == -INFINITY) continue;
+        if (l[q] > mx) {
+          sum = (mx == -INFINITY ? 0.f : sum * expf(mx - l[q])) + 1.f;
+          mx = l[q];
+        } else {
+          sum += expf(l[q] - mx);
+        }
       }
-      if (!ep_sync()) return;
-      if (warp == 0) {
-        const int rr = r + 8 * hf;
-        if (rr < rows) {
-          const int m = rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G, hq = h * a.G + g;
-          const float lse_v = hf ? lse1 : lse0;
+    }
+  }
+  const float my_lse = mx == -INFINITY ? -INFINITY : mx + logf(sum);
+  for (int r0 = 0; r0 < rows; r0 += 4) {
+    float acc[4][VEC];
 #pragma unroll
-          for (int dn = 0; dn < DN; ++dn) {
-            float v0 = o[dn][2 * hf], v1 = o[dn][2 * hf + 1];
+    for (int q = 0; q < 4; ++q)
 #pragma unroll
-            for (int w = 0; w < kConsumerWarps - 1; ++w) {
-              const float2 p = *reinterpret_cast<const float2 *>(&merge[(w * 8 + r) * D + dn * 8 + 2 * c]);
-              v0 += p.x;
-              v1 += p.y;
-            }
-            const int d = dn * 8 + 2 * c;
-            if (kind == 0) {
-              uint32_t *dst = reinterpret_cast<uint32_t *>(
-                  reinterpret_cast<uint16_t *>(a.out) + ((size_t)(b * a.q_len + t) * a.Hq + hq) * D + d);
-              *dst = pack2<kBf16>(v0, v1);
-            } else {
-              *reinterpret_cast<float2 *>(a.o_part + (((size_t)blockIdx.x * 2 + slot) * kRowsPerTile + rr) * D + d) =
-                  make_float2(v0, v1);
-            }
-          }
-          if (c == 0) {
-            if (kind == 0) {
-              if (a.lse != nullptr) a.lse[((size_t)b * a.Hq + hq) * a.q_len + t] = lse_v;
-            } else {
-              a.lse_part[((size_t)blockIdx.x * 2 + slot) * kRowsPerTile + rr] = lse_v;
-            }
+      for (int v = 0; v < VEC; ++v) acc[q][v] = 0.f;
+    float lse_q[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) lse_q[q] = __shfl_sync(0xffffffffu, my_lse, (r0 + q) & 31);
+    for (int i = 0; i < n; ++i) {
+      const size_t sl = slot_of(i);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int rr = r0 + q;
+        if (rr < rows && lse_q[q] != -INFINITY) {
+          const float w = expf(__ldcg(a.lse_part + sl * kRowsPerTile + rr) - lse_q[q]);
+          const float *src = a.o_part + (sl * kRowsPerTile + rr) * D + col;
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) acc[q][v] += w * __ldcg(src + v);
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int rr = r0 + q;
+      if (rr < rows) {
+        const int m = sg.rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G, hq = sg.h * a.G + g;
+        store_out_vec<D, kBf16>(a, sg.b, t, hq, col, acc[q]);
+        if (lane == 0 && a.lse != nullptr) a.lse[((size_t)sg.b * a.Hq + hq) * a.q_len + t] = lse_q[q];
+      }
+    }
+  }
+  if (lane == 0) a.counters[unit] = 0ull;  // every piece has arrived; leave it clean
+}
+
+template <int D, bool kBf16>
+__device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
+  constexpr int VEC = D / 32;
+  constexpr int T = block_tokens(D);
+  constexpr uint32_t KV_BYTES = (uint32_t)T * D * 2;
+  constexpr float NEG_INF = -INFINITY;
+  const uint32_t ring = smem_addr(smem + smem_ring_off());
+  JobSlot *jobs = reinterpret_cast<JobSlot *>(smem + smem_jobs_off(D));
+  const int HR = a.Hkv * a.RT;
+
+  // Units of rows with L_b = 0 hold no KV block; one CTA per unit writes
+  // their empty result.
+  if (a.schedule == MXA_SCHED_BALANCED) {
+    for (int u = blockIdx.x; u < a.units; u += gridDim.x)
+      if (clamp_len(a.seqlens[u / HR], a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, lane);
+  } else if (blockIdx.x % a.splits == 0) {
+    const int u = blockIdx.x / a.splits;
+    if (clamp_len(a.seqlens[u / HR], a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, lane);
+  }
+
+  const int col = lane * VEC;
+  for (int jn = 0;; ++jn) {
+    const int j = jn % kJobs, jk = jn / kJobs;
+    if (!warp_wait_bounded(bar_addr(smem, D, B_JOBFULL(j)), jk & 1, &g_mxa_err, kErrWaitFull, lane)) return;
+    const SegmentDesc sg = jobs[j].seg;
+    if (sg.kind < 0) return;
+    const int stage = jobs[j].stage;
+    const uint32_t sbase = ring + (uint32_t)stage * (2 * KV_BYTES);
+    const int rows = min(kRowsPerTile, a.M - sg.rt * kRowsPerTile);
+    const int unit = (sg.b * a.Hkv + sg.h) * a.RT + sg.rt;
+    const int slot = sg.kind - 1;  // partial slot (kind 1 -> head slot 0, kind 2 -> tail slot 1)
+
+    // statistics of row `lane`: the four warps' (m, l) merged
+    float wgt[kMathWarps];
+    float my_lse = NEG_INF;
+#pragma unroll
+    for (int w = 0; w < kMathWarps; ++w) wgt[w] = 0.f;
+    {
+      const int row = lane < rows ? lane : 0;  // every lane computes; rows' lanes are used
+      float mw[kMathWarps], lw[kMathWarps];
+      float Mx = NEG_INF;
+#pragma unroll
+      for (int w = 0; w < kMathWarps; ++w) {
+        mw[w] = jobs[j].ml[w][row][0];
+        lw[w] = jobs[j].ml[w][row][1];
+        Mx = fmaxf(Mx, mw[w]);
+      }
+      float Lx = 0.f;
+#pragma unroll
+      for (int w = 0; w < kMathWarps; ++w) {
+        wgt[w] = mw[w] != NEG_INF ? ex2(mw[w] - Mx) : 0.f;
+        Lx += wgt[w] * lw[w];
+      }
+      const float inv = Lx > 0.f ? 1.f / Lx : 0.f;
+#pragma unroll
+      for (int w = 0; w < kMathWarps; ++w) wgt[w] *= inv;
+      my_lse = Lx > 0.f ? (Mx + log2f(Lx)) * kLn2 : NEG_INF;
+    }
+    for (int rr = 0; rr < rows; ++rr) {
+      float acc[VEC];
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+#pragma unroll
+      for (int w = 0; w < kMathWarps; ++w) {
+        const float wg = __shfl_sync(0xffffffffu, wgt[w], rr);
+        if (wg != 0.f) {
+          const uint32_t addr = handoff_addr<D>(sbase, w, rr, col);
+          if constexpr (VEC == 4) {
+            float4 v;
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+            acc[0] += wg * v.x; acc[1] += wg * v.y; acc[2] += wg * v.z; acc[3] += wg * v.w;
+          } else {
+            float2 v;
+            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+            acc[0] += wg * v.x; acc[1] += wg * v.y;
           }
         }
+      }
+      const float lse = __shfl_sync(0xffffffffu, my_lse, rr);
+      const int m = sg.rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G, hq = sg.h * a.G + g;
+      if (sg.kind == 0) {
+        store_out_vec<D, kBf16>(a, sg.b, t, hq, col, acc);
+        if (lane == 0 && a.lse != nullptr) a.lse[((size_t)sg.b * a.Hq + hq) * a.q_len + t] = lse;
+      } else {
+        float *dst = a.o_part + (((size_t)blockIdx.x * 2 + slot) * kRowsPerTile + rr) * D + col;
+        if constexpr (VEC == 4) {
+          *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        } else {
+          *reinterpret_cast<float2 *>(dst) = make_float2(acc[0], acc[1]);
+        }
+        if (lane == 0) a.lse_part[((size_t)blockIdx.x * 2 + slot) * kRowsPerTile + rr] = lse;
+      }
+    }
+    // Give the stage back to the producer and the hand-off slot to the math
+    // warps.  This warp only read the stage; the math warps fenced their
+    // generic writes to it before handing it over.
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_cnt(bar_addr(smem, D, B_EMPTY(stage)), kMathWarps);
+      mbar_arrive(bar_addr(smem, D, B_JOBEMPTY(j)));
+    }
+    if (sg.kind != 0) {  // a piece of a split unit: the last piece to arrive merges them all
+      __threadfence();
+      __syncwarp();
+      if (arrive_and_check_last(a, unit, sg.n_pieces, lane)) {
+        __threadfence();
+        merge_pieces<D, kBf16>(a, sg, rows, unit, lane);
       }
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// The split kernel: CTA prologue (find this CTA's range of KV blocks), then
-// warp-specialised producer / consumers.
+// The split kernel
 // ---------------------------------------------------------------------------
 template <int D, bool kBf16>
 __global__ void __launch_bounds__(kThreads, 2)
-    mxa_split_kernel(const __grid_constant__ TmapPair tm, const DecodeArgs a) {
+    mxa_split_kernel(const __grid_constant__ TmapPair tm, const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  constexpr int T = block_tokens(D);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if ((smem_addr(smem) & 1023u) != 0) {  // the 128-byte swizzle needs 1024-byte aligned stages
     if (tid == 0) atomicOr(&g_mxa_err, kErrAlign);
     return;
   }
-  const uint32_t bar0 = smem_addr(smem + smem_bar_off(D));
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar0 + 8u * s, 1);                          // full: producer arrival + bytes
-      mbar_init(bar0 + 8u * (kStages + s), kConsumerWarps);  // empty: one arrival per consumer warp
+      mbar_init(bar_addr(smem, D, B_FULL(s)), 1);            // producer arrival + bytes
+      mbar_init(bar_addr(smem, D, B_EMPTY(s)), kMathWarps);  // one arrival per math warp
     }
-    mbar_init(bar0 + 8u * (2 * kStages), 1);                 // qfull
-    mbar_init(bar0 + 8u * (2 * kStages + 1), kConsumerWarps);// qempty
-    mbar_init(bar0 + 8u * (2 * kStages + 2), kConsumerWarps);// epilogue sync
+    mbar_init(bar_addr(smem, D, B_QFULL), 1);
+    mbar_init(bar_addr(smem, D, B_QEMPTY), kMathWarps);
+    for (int j = 0; j < kJobs; ++j) {
+      mbar_init(bar_addr(smem, D, B_JOBFULL(j)), kMathWarps);
+      mbar_init(bar_addr(smem, D, B_JOBEMPTY(j)), 1);
+    }
     fence_mbar_init();
   }
-
-  const int HR = a.Hkv * a.RT;
-  long long *info = reinterpret_cast<long long *>(smem + smem_ml_off(D));  // scratch until the first epilogue
-  if (a.schedule == MXA_SCHED_BALANCED) {
-    // Blocks per row, prefix-summed in shared memory (the ring is still free).
-    int *scan = reinterpret_cast<int *>(smem + smem_ring_off());
-    int *part = scan + kMaxBalancedRows;
-    for (int b = tid; b < a.B; b += kThreads)
-      scan[b] = (clamp_len(a.seqlens[b], a.max_seqlen_k) + T - 1) / T;
-    __syncthreads();
-    const int chunk = (a.B + kThreads - 1) / kThreads;
-    const int lo = min(tid * chunk, a.B), hi = min(lo + chunk, a.B);
-    int sum = 0;
-    for (int i = lo; i < hi; ++i) sum += scan[i];
-    part[tid] = sum;
-    __syncthreads();
-    if (tid == 0) {
-      int run = 0;
-      for (int i = 0; i < kThreads; ++i) {
-        const int v = part[i];
-        part[i] = run;
-        run += v;
-      }
-      info[7] = run;
-    }
-    __syncthreads();
-    int run = part[tid];
-    for (int i = lo; i < hi; ++i) {
-      run += scan[i];
-      scan[i] = run;  // inclusive prefix
-    }
-    __syncthreads();
-    if (tid == 0) {
-      const long long NB = (long long)HR * info[7];
-      const long long P = NB == 0 ? 1 : (NB + a.grid - 1) / a.grid;
-      const long long x0 = (long long)blockIdx.x * P;
-      long long b0 = 0, hr0 = 0, blk0 = 0, rem = 0;
-      if (x0 < NB) {
-        int lo_b = 0, hi_b = a.B - 1;  // first row whose blocks end past x0
-        while (lo_b < hi_b) {
-          const int mid = (lo_b + hi_b) >> 1;
-          if ((long long)HR * scan[mid] > x0) hi_b = mid; else lo_b = mid + 1;
-        }
-        b0 = lo_b;
-        const long long pre = b0 > 0 ? scan[b0 - 1] : 0;
-        const long long nb = scan[b0] - pre;
-        const long long off = x0 - (long long)HR * pre;
-        hr0 = off / nb;
-        blk0 = off % nb;
-        rem = P < NB - x0 ? P : NB - x0;
-      }
-      info[0] = b0; info[1] = hr0; info[2] = blk0; info[3] = rem; info[4] = x0; info[5] = P;
-    }
-    fence_proxy_async_smem();  // generic writes above precede TMA writes to the ring
-    __syncthreads();
-  } else {
-    if (tid == 0) {
-      const int u = blockIdx.x / a.splits, si = blockIdx.x % a.splits;
-      const int b = u / HR, hr = u % HR;
-      const int L = clamp_len(a.seqlens[b], a.max_seqlen_k);
-      const int nb = (L + T - 1) / T;
-      const int beg = si * a.chunk_blocks, end = min(beg + a.chunk_blocks, nb);
-      info[0] = b; info[1] = hr; info[2] = beg; info[3] = end > beg ? end - beg : 0;
-      info[4] = 0; info[5] = 1;
-    }
-    __syncthreads();
-  }
-
-  if (warp == kConsumerWarps) {
-    Walk<D> w;
-    w.b = (int)info[0];
-    w.hr = (int)info[1];
-    w.blk = (int)info[2];
-    w.remaining = info[3];
-    w.x = info[4];
-    w.per_cta = info[5];
-    w.L = 0;
-    w.nb = 0;
-    if (w.remaining > 0) walk_load_row(w, a);
-    producer_warp<D, kBf16>(tm, a, w, smem, lane);
-    return;
-  }
-
-  // Rows with L_b = 0 belong to no KV block; one CTA per such unit writes
-  // its empty result.
-  if (a.schedule == MXA_SCHED_BALANCED) {
-    for (int u = blockIdx.x; u < a.units; u += a.grid) {
-      const int b = u / HR;
-      if (clamp_len(a.seqlens[b], a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, tid);
-    }
-  } else if (blockIdx.x % a.splits == 0) {
-    const int u = blockIdx.x / a.splits;
-    if (clamp_len(a.seqlens[u / HR], a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, tid);
-  }
-  consumer_warps<D, kBf16>(a, smem, warp, lane);
-  grid_launch_dependents();
-}
-
-// ---------------------------------------------------------------------------
-// Merge of units split across CTAs (balanced or uniform schedule): the
-// log-sum-exp reduce of the split results.  One CTA per unit.
-// ---------------------------------------------------------------------------
-template <int D, bool kBf16>
-__global__ void __launch_bounds__(128) mxa_merge_kernel(const MergeArgs a) {
-  grid_dependency_wait();  // the split kernel's writes are visible past this point
-  const int u = blockIdx.x;
-  const int2 mt = a.meta[u];
-  if (mt.y <= mt.x) return;  // the unit was finished by one CTA
-  if (mt.x < 0 || mt.y >= a.grid) return;  // not written by this call (only after a failed wait)
-  const int n = mt.y - mt.x + 1;
-  const int rt = u % a.RT, hr = u / a.RT, h = hr % a.Hkv, b = hr / a.Hkv;
-  const int rows = min(kRowsPerTile, a.M - rt * kRowsPerTile);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // the unit's pieces: the tail slot of its first CTA, then the head slots
-  // of the following CTAs
-  auto slot = [&](int i) { return i == 0 ? (size_t)mt.x * 2 + 1 : (size_t)(mt.x + i) * 2; };
-  __shared__ float s_lse[kRowsPerTile];
-
-  for (int rr = warp; rr < rows; rr += 4) {
-    float mx = -INFINITY;
-    for (int i = lane; i < n; i += 32) mx = fmaxf(mx, a.lse_part[slot(i) * kRowsPerTile + rr]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float sum = 0.f;
-    if (mx != -INFINITY)
-      for (int i = lane; i < n; i += 32) sum += expf(a.lse_part[slot(i) * kRowsPerTile + rr] - mx);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float lse = mx == -INFINITY ? -INFINITY : mx + logf(sum);
-    if (lane == 0) {
-      s_lse[rr] = lse;
-      if (a.lse != nullptr) {
-        const int m = rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G;
-        a.lse[((size_t)b * a.Hq + (size_t)h * a.G + g) * a.q_len + t] = lse;
-      }
-    }
-  }
   __syncthreads();
-  for (int idx = tid; idx < rows * (D / 4); idx += 128) {
-    const int rr = idx / (D / 4), d = (idx % (D / 4)) * 4;
-    const float lse = s_lse[rr];
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (lse != -INFINITY) {
-      for (int i = 0; i < n; ++i) {
-        const size_t sl = slot(i);
-        const float wgt = expf(a.lse_part[sl * kRowsPerTile + rr] - lse);
-        const float4 v = *reinterpret_cast<const float4 *>(a.o_part + (sl * kRowsPerTile + rr) * D + d);
-        acc.x += wgt * v.x;
-        acc.y += wgt * v.y;
-        acc.z += wgt * v.z;
-        acc.w += wgt * v.w;
-      }
-    }
-    const int m = rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G;
-    uint2 packed = make_uint2(pack2<kBf16>(acc.x, acc.y), pack2<kBf16>(acc.z, acc.w));
-    *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(a.out) +
-                               ((size_t)(b * a.q_len + t) * a.Hq + (size_t)h * a.G + g) * D + d) = packed;
+  if (warp == kProducerWarp) {
+    producer_warp<D, kBf16>(tm, a, smem, lane);
+  } else if (warp == kEpilogueWarp) {
+    epilogue_warp<D, kBf16>(a, smem, lane);
+  } else {
+    math_warps<D, kBf16>(a, smem, warp, lane);
   }
 }
 
@@ -761,6 +939,8 @@ __global__ void __launch_bounds__(128)
 // Host side: tensor maps and launches
 // ===========================================================================
 #include <cudaTypedefs.h>
+
+#include <atomic>
 #include <mutex>
 
 namespace mxa {
@@ -781,6 +961,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// 3-D map {D, Hkv, pool tokens} of a K or V pool; box {64 elements, 1 head,
+// box_tokens tokens}, 128-byte swizzle, zero fill out of bounds.
 bool encode_kv_map(CUtensorMap *m, const void *base, int D, int Hkv, long long pool_tokens,
                    int box_tokens, bool bf16) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
@@ -805,6 +987,14 @@ cudaError_t prepare_split_kernel(int device) {
   cudaError_t e = cudaFuncSetAttribute(mxa_split_kernel<D, kBf16>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_total(D));
   if (e == cudaSuccess && device >= 0 && device < kMaxDevices) done[device] = true;
+  return e;
+}
+
+// Epoch of a launch: tags the arrival counters of split units (never 0).
+uint32_t next_epoch() {
+  static std::atomic<uint32_t> counter{0};
+  uint32_t e = ++counter;
+  if (e == 0) e = ++counter;
   return e;
 }
 
@@ -838,19 +1028,17 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
   a.scale_log2 = L.scale * 1.4426950408889634f;
   a.causal = L.causal;
   a.schedule = plan.schedule;
-  a.grid = plan.grid;
   a.splits = plan.num_splits;
   const int max_blocks = (p.max_seqlen_k + T - 1) / T;
-  a.chunk_blocks = plan.schedule == MXA_SCHED_UNIFORM
-                       ? (max_blocks + plan.num_splits - 1) / plan.num_splits
-                       : 1;
+  a.chunk_blocks = plan.schedule == MXA_SCHED_UNIFORM ? (max_blocks + plan.num_splits - 1) / plan.num_splits : 1;
   if (a.chunk_blocks < 1) a.chunk_blocks = 1;
   a.units = plan.units;
+  a.epoch = next_epoch();
   if (plan.workspace_bytes > 0) {
     uint8_t *ws = static_cast<uint8_t *>(L.workspace);
-    a.meta = reinterpret_cast<int2 *>(ws);
-    a.lse_part = reinterpret_cast<float *>(ws + ws_meta_bytes(plan.units));
-    a.o_part = reinterpret_cast<float *>(ws + ws_meta_bytes(plan.units) + ws_lse_bytes(plan.grid));
+    a.counters = reinterpret_cast<unsigned long long *>(ws);
+    a.lse_part = reinterpret_cast<float *>(ws + ws_count_bytes(plan.units));
+    a.o_part = reinterpret_cast<float *>(ws + ws_count_bytes(plan.units) + ws_lse_bytes(plan.grid));
   }
 
   TmapPair tm;
@@ -860,35 +1048,7 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
     return MXA_ERR_CUDA;
 
   mxa_split_kernel<D, kBf16><<<plan.grid, kThreads, smem_total(D), stream>>>(tm, a);
-  if (cudaGetLastError() != cudaSuccess) return MXA_ERR_CUDA;
-
-  if (plan.needs_combine) {
-    MergeArgs m{};
-    m.meta = a.meta;
-    m.lse_part = a.lse_part;
-    m.o_part = a.o_part;
-    m.out = L.out;
-    m.lse = L.lse;
-    m.q_len = a.q_len;
-    m.Hq = a.Hq;
-    m.Hkv = a.Hkv;
-    m.G = a.G;
-    m.M = a.M;
-    m.RT = a.RT;
-    m.grid = plan.grid;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)plan.units);
-    cfg.blockDim = dim3(128);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the launch with the split kernel's tail
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, mxa_merge_kernel<D, kBf16>, m) != cudaSuccess) return MXA_ERR_CUDA;
-  }
-  return MXA_OK;
+  return cudaGetLastError() == cudaSuccess ? MXA_OK : MXA_ERR_CUDA;
 }
 
 }  // namespace

@@ -18,37 +18,27 @@ struct alignas(64) TmapPair {
 };
 
 struct DecodeArgs {
-  const void *q;            // [B, q_len, Hq, D]
+  const void *q;               // [B, q_len, Hq, D]
   const int32_t *block_table;  // [B, mpps] (unused when contiguous)
-  const int32_t *seqlens;   // [B]
-  void *out;                // [B, q_len, Hq, D]
-  float *lse;               // [B, Hq, q_len] or null
-  int2 *meta;               // [units]: first and last CTA holding a piece of the unit
-  float *lse_part;          // [grid][2][16]
-  float *o_part;            // [grid][2][16][D]
+  const int32_t *seqlens;      // [B]
+  void *out;                   // [B, q_len, Hq, D]
+  float *lse;                  // [B, Hq, q_len] or null
+  unsigned long long *counters;  // [units]: epoch-tagged arrivals of split units
+  float *lse_part;             // [grid][2][16]
+  float *o_part;               // [grid][2][16][D]
   int B, q_len, Hq, Hkv, G, M, RT;
-  int page_size;            // slots per page (row capacity when contiguous)
-  int mpps;                 // block-table row stride
+  int page_size;               // slots per page (row capacity when contiguous)
+  int mpps;                    // block-table row stride
   int contiguous;
   int max_seqlen_k;
-  int box_tokens;           // tokens per TMA box
-  float scale_log2;         // scale * log2(e)
+  int box_tokens;              // tokens per TMA box
+  float scale_log2;            // scale * log2(e)
   int causal;
-  int schedule;             // mxa_schedule_t
-  int grid;
-  int splits;               // UNIFORM: splits per unit
-  int chunk_blocks;         // UNIFORM: blocks per split
+  int schedule;                // mxa_schedule_t
+  int splits;                  // UNIFORM: splits per unit
+  int chunk_blocks;            // UNIFORM: blocks per split
   int units;
-};
-
-struct MergeArgs {
-  const int2 *meta;
-  const float *lse_part;
-  const float *o_part;
-  void *out;
-  float *lse;
-  int q_len, Hq, Hkv, G, M, RT;
-  int grid;  // CTAs of the split kernel: metadata outside [0, grid) is ignored
+  unsigned int epoch;          // tags this launch's arrival counts
 };
 
 // Everything launch_decode needs; pointers are device pointers.
@@ -64,7 +54,7 @@ struct DecodeLaunch {
   int causal;
 };
 
-// Launch the split kernel and, when the plan needs it, the merge kernel.
+// Launch the split kernel (split units are merged inside it).
 mxa_status_t launch_decode(const DecodeLaunch &L, cudaStream_t stream);
 
 // Launch the uniform-layout combine of mxa_combine().

@@ -106,7 +106,7 @@ typedef struct {
   int block_tokens;      /* KV tokens per pipeline stage */
   int ctas_per_sm;       /* resident CTAs per SM the plan assumed */
   int sm_count;          /* SMs the plan assumed */
-  int needs_combine;     /* 1 if a combine pass follows the split kernel */
+  int needs_combine;     /* 1 if units may be split across CTAs and merged (needs the workspace) */
   size_t workspace_bytes;/* device scratch the run needs (0 if none) */
 } mxa_plan_t;
 
