@@ -134,7 +134,7 @@ __device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
 // (still unused) ring by this warp alone.  UNIFORM: block range
 // [si * chunk, (si + 1) * chunk) of unit blockIdx.x / splits.
 template <int D>
-__device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane) {
+__device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cursor &tail, bool &has_tail) {
   constexpr int T = block_tokens(D);
   const int HR = a.Hkv * a.RT;
   Cursor c;
@@ -144,6 +144,8 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane) {
   c.x = 0;
   c.per_cta = 1;
   c.L = c.nb = c.L_next = 0;
+  has_tail = false;
+  tail = c;
   if (a.schedule == MXA_SCHED_UNIFORM) {
     const int u = blockIdx.x / a.splits, si = blockIdx.x % a.splits;
     c.b = u / HR;
@@ -200,6 +202,35 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane) {
     c.nb = (int)nb;  // from the scan: the length itself is first needed later
     c.L = clamp_len(a.seqlens[c.b], a.max_seqlen_k);
     c.L_next = c.b + 1 < a.B ? a.seqlens[c.b + 1] : 0;
+
+    // If the range ends inside a unit that starts within it (a tail piece),
+    // that piece is handled first: its other pieces are then also done early
+    // in their CTAs, and the unit's merge overlaps streaming instead of
+    // lengthening the end of the kernel.
+    const long long xl = x0 + c.remaining - 1;
+    int lb = lo_b, hb = a.B - 1;
+    while (lb < hb) {
+      const int mid = (lb + hb) >> 1;
+      if ((long long)HR * scan[mid] > xl) hb = mid; else lb = mid + 1;
+    }
+    const long long pre_l = lb > 0 ? scan[lb - 1] : 0;
+    const long long nb_l = scan[lb] - pre_l;
+    const long long off_l = xl - (long long)HR * pre_l;
+    const int hr_l = (int)(off_l / nb_l), blk_l = (int)(off_l % nb_l);
+    const long long x_t = xl - blk_l;  // flattened index of that unit's first block
+    if (blk_l + 1 < nb_l && x_t > x0) {
+      tail.b = lb;
+      tail.hr = hr_l;
+      tail.blk = 0;
+      tail.remaining = blk_l + 1;
+      tail.x = x_t;
+      tail.per_cta = c.per_cta;
+      tail.nb = (int)nb_l;
+      tail.L = clamp_len(a.seqlens[lb], a.max_seqlen_k);
+      tail.L_next = 0;
+      has_tail = true;
+      c.remaining = x_t - x0;
+    }
   }
   __syncwarp();
   fence_proxy_async_smem();  // these generic writes precede the TMA writes to the ring
@@ -233,7 +264,17 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
     prefetch_tmap(&tm.k);
     prefetch_tmap(&tm.v);
   }
-  Cursor cur = cursor_start<D>(a, smem, lane);
+  Cursor tail;
+  bool has_tail;
+  Cursor cur = cursor_start<D>(a, smem, lane, tail, has_tail);
+  auto more = [&]() { return has_tail || (cur.remaining > 0 && cur.nb > 0); };
+  auto take = [&]() {
+    if (has_tail) {
+      has_tail = false;
+      return cursor_take<D>(tail, a);
+    }
+    return cursor_take<D>(cur, a);
+  };
 
   // Publish a segment to the math warps: its descriptor and its Q tile.
   auto issue_q = [&](const SegmentDesc &s) {
@@ -264,8 +305,8 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
   int it = 0;     // KV stages issued
   int seg_k = 0;  // segments published
   bool ok = true;
-  if (cur.remaining > 0 && cur.nb > 0) {
-    SegmentDesc seg = cursor_take<D>(cur, a);
+  if (more()) {
+    SegmentDesc seg = take();
     Window win;
     load_window(seg, win);
     if (!warp_wait_bounded(qempty, 1, &g_mxa_err, kErrWaitQ, lane)) ok = false;  // first use: free
@@ -274,14 +315,9 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
       ++seg_k;
     }
     while (ok) {
-      const bool have_next = cur.remaining > 0 && cur.nb > 0;
+      bool have_next = false, next_known = false, q_next = false;
       SegmentDesc nseg;
       Window nwin;
-      bool q_next = false;
-      if (have_next) {
-        nseg = cursor_take<D>(cur, a);
-        load_window(nseg, nwin);  // its latency hides behind this segment's stages
-      }
       for (int blk = seg.blk_beg; blk < seg.blk_end; ++blk) {
         const int s = it % kStages;
         const int k = it / kStages;
@@ -321,6 +357,16 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
                       bar_addr(smem, D, B_FULL(s)));
         }
         ++it;
+        // Find the next segment once this one's first stage is on its way
+        // (its loads then hide behind this segment's stages).
+        if (!next_known) {
+          next_known = true;
+          have_next = more();
+          if (have_next) {
+            nseg = take();
+            load_window(nseg, nwin);
+          }
+        }
         // publish the next segment as soon as the math warps hold this one's Q
         if (have_next && !q_next) {
           bool free_slot = false;
@@ -671,70 +717,68 @@ __device__ __forceinline__ bool arrive_and_check_last(const DecodeArgs &a, int u
   }
 }
 
-// Merge the n pieces of a split unit with the log-sum-exp identity:
-// LSE = ln sum_i exp(lse_i), O = sum_i exp(lse_i - LSE) O_i.  The pieces are
-// the tail slot of the first CTA and the head slots of the following ones.
-// Lane r < rows owns the statistics of packed row r; every lane owns D / 32
-// output columns of every row.  Loads of one round are independent, so a
-// merge costs a few memory round trips whatever the number of rows.
+// Merge the n pieces of a split unit with the log-sum-exp identity,
+// LSE = ln sum_i exp(lse_i) and O = sum_i exp(lse_i - LSE) O_i, in one pass
+// with a running maximum per row.  The pieces are the tail slot of the
+// first CTA and the head slots of the following ones.  Every lane owns
+// D / 32 output columns; the loads of a batch of 4 pieces x 4 rows are
+// independent, so a batch costs one memory round trip.
 template <int D, bool kBf16>
 __device__ void merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int rows, int unit, int lane) {
   constexpr int VEC = D / 32;
+  constexpr int PB = 4, RB = 4;  // pieces and rows per batch
   const int n = sg.n_pieces, cf = sg.c_first;
   auto slot_of = [&](int i) -> size_t { return i == 0 ? (size_t)cf * 2 + 1 : (size_t)(cf + i) * 2; };
   const int col = lane * VEC;
-  // statistics of row `lane`, one pass with a running maximum (loads of a
-  // batch of 8 pieces are issued together)
-  float mx = -INFINITY, sum = 0.f;
-  {
-    const bool mine = lane < rows;  // all lanes run the loop; only rows' lanes load
-    for (int i0 = 0; i0 < n; i0 += 8) {
-      float l[8];
+  for (int r0 = 0; r0 < rows; r0 += RB) {
+    float m[RB], ssum[RB], acc[RB][VEC];
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        l[q] = (mine && i0 + q < n) ? __ldcg(a.lse_part + slot_of(i0 + q) * kRowsPerTile + lane) : -INFINITY;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (l[q] == -INFINITY) continue;
-        if (l[q] > mx) {
-          sum = (mx == -INFINITY ? 0.f : sum * expf(mx - l[q])) + 1.f;
-          mx = l[q];
-        } else {
-          sum += expf(l[q] - mx);
-        }
-      }
-    }
-  }
-  const float my_lse = mx == -INFINITY ? -INFINITY : mx + logf(sum);
-  for (int r0 = 0; r0 < rows; r0 += 4) {
-    float acc[4][VEC];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
+    for (int q = 0; q < RB; ++q) {
+      m[q] = -INFINITY;
+      ssum[q] = 0.f;
 #pragma unroll
       for (int v = 0; v < VEC; ++v) acc[q][v] = 0.f;
-    float lse_q[4];
+    }
+    for (int i0 = 0; i0 < n; i0 += PB) {
+      float l[PB][RB], o[PB][RB][VEC];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) lse_q[q] = __shfl_sync(0xffffffffu, my_lse, (r0 + q) & 31);
-    for (int i = 0; i < n; ++i) {
-      const size_t sl = slot_of(i);
+      for (int p = 0; p < PB; ++p) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int rr = r0 + q;
-        if (rr < rows && lse_q[q] != -INFINITY) {
-          const float w = expf(__ldcg(a.lse_part + sl * kRowsPerTile + rr) - lse_q[q]);
-          const float *src = a.o_part + (sl * kRowsPerTile + rr) * D + col;
+        for (int q = 0; q < RB; ++q) {
+          const bool live = i0 + p < n && r0 + q < rows;
+          const size_t base = live ? slot_of(i0 + p) * kRowsPerTile + r0 + q : 0;
+          l[p][q] = live ? __ldcg(a.lse_part + base) : -INFINITY;
 #pragma unroll
-          for (int v = 0; v < VEC; ++v) acc[q][v] += w * __ldcg(src + v);
+          for (int v = 0; v < VEC; ++v) o[p][q][v] = live ? __ldcg(a.o_part + base * D + col + v) : 0.f;
+        }
+      }
+#pragma unroll
+      for (int p = 0; p < PB; ++p) {
+#pragma unroll
+        for (int q = 0; q < RB; ++q) {
+          if (l[p][q] == -INFINITY) continue;  // an empty piece carries no weight
+          const float mn = fmaxf(m[q], l[p][q]);
+          const float keep = m[q] == -INFINITY ? 0.f : expf(m[q] - mn);
+          const float w = expf(l[p][q] - mn);
+          ssum[q] = ssum[q] * keep + w;
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) acc[q][v] = acc[q][v] * keep + w * o[p][q][v];
+          m[q] = mn;
         }
       }
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < RB; ++q) {
       const int rr = r0 + q;
       if (rr < rows) {
-        const int m = sg.rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G, hq = sg.h * a.G + g;
-        store_out_vec<D, kBf16>(a, sg.b, t, hq, col, acc[q]);
-        if (lane == 0 && a.lse != nullptr) a.lse[((size_t)sg.b * a.Hq + hq) * a.q_len + t] = lse_q[q];
+        const float inv = ssum[q] > 0.f ? 1.f / ssum[q] : 0.f;
+        float out_v[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) out_v[v] = acc[q][v] * inv;
+        const float lse = m[q] == -INFINITY ? -INFINITY : m[q] + logf(ssum[q]);
+        const int mrow = sg.rt * kRowsPerTile + rr, t = mrow / a.G, g = mrow % a.G, hq = sg.h * a.G + g;
+        store_out_vec<D, kBf16>(a, sg.b, t, hq, col, out_v);
+        if (lane == 0 && a.lse != nullptr) a.lse[((size_t)sg.b * a.Hq + hq) * a.q_len + t] = lse;
       }
     }
   }
