@@ -18,7 +18,10 @@ constexpr int kMaxThreadsPerSm = 2048;
 constexpr int kMaxBalancedRows = 16384;                 // balanced schedule scans B rows in smem
 
 // KV tokens per pipeline stage: every stage carries T x D elements of K and
-// of V (16 KiB each in 16-bit types), so T = 8192 / D.
+// of V (16 KiB each in 16-bit types), so T = 8192 / D.  Three stages per CTA
+// and two CTAs per SM keep 192 KiB of loads in flight per SM, which is what
+// B200's HBM needs at its loaded latency of several microseconds; two CTAs
+// also let one stream while the other starts up or finishes.
 constexpr int block_tokens(int D) { return 8192 / D; }
 
 constexpr size_t stage_bytes(int D) { return (size_t)2 * block_tokens(D) * D * 2; }

@@ -324,23 +324,11 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
         const int tok0 = blk * T;
         const int valid = min(T, seg.L - tok0);
         const int nbox = (valid + bt - 1) / bt;
-        const int n_ops = nbox * CH * 2;
-        const int box = lane / (CH * 2);
-        const int ch = (lane / 2) % CH;
-        const int kv = lane & 1;
-        const int tok = tok0 + box * bt;
-        int page = 0;
-        if (!a.contiguous) {
-          if (tok0 / ps - win.base >= 32) {  // slide the window by 32 pages
-            win.base += 32;
-            win.wa = win.wb;
-            win.wb = bt_entry(a, seg.b, win.base + 32 + lane, a.mpps);
-          }
-          const int idx = tok / ps - win.base;
-          const int src = idx & 31;
-          const int va = __shfl_sync(0xffffffffu, win.wa, src);
-          const int vb = __shfl_sync(0xffffffffu, win.wb, src);
-          page = idx < 32 ? va : vb;
+        const int n_ops = nbox * CH * 2;  // one TMA box per (page box, 64-column chunk, K or V)
+        if (!a.contiguous && tok0 / ps - win.base >= 32) {  // slide the window by 32 pages
+          win.base += 32;
+          win.wa = win.wb;
+          win.wb = bt_entry(a, seg.b, win.base + 32 + lane, a.mpps);
         }
         if (!warp_wait_bounded(bar_addr(smem, D, B_EMPTY(s)), (k & 1) ^ 1, &g_mxa_err, kErrWaitEmpty,
                                lane)) {
@@ -349,12 +337,27 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
         }
         if (lane == 0) mbar_arrive_expect_tx(bar_addr(smem, D, B_FULL(s)), (uint32_t)nbox * bt * D * 2 * 2);
         __syncwarp();
-        if (lane < n_ops) {
-          const int row = a.contiguous ? seg.b * ps + tok : page * ps + tok % ps;
-          const uint32_t dst = ring + (uint32_t)s * (2 * KV_BYTES) + (uint32_t)kv * KV_BYTES +
-                               (uint32_t)ch * (T * 128) + (uint32_t)(box * bt) * 128;
-          tma_load_3d(dst, kv ? (const void *)&tm.v : (const void *)&tm.k, ch * 64, seg.h, row,
-                      bar_addr(smem, D, B_FULL(s)));
+        for (int op0 = 0; op0 < n_ops; op0 += 32) {  // all lanes take part in every shuffle
+          const int op = op0 + lane;
+          const int box = op / (CH * 2);
+          const int ch = (op / 2) % CH;
+          const int kv = op & 1;
+          const int tok = tok0 + box * bt;
+          int page = 0;
+          if (!a.contiguous) {
+            const int idx = tok / ps - win.base;
+            const int src = idx & 31;
+            const int va = __shfl_sync(0xffffffffu, win.wa, src);
+            const int vb = __shfl_sync(0xffffffffu, win.wb, src);
+            page = idx < 32 ? va : vb;
+          }
+          if (op < n_ops) {
+            const int row = a.contiguous ? seg.b * ps + tok : page * ps + tok % ps;
+            const uint32_t dst = ring + (uint32_t)s * (2 * KV_BYTES) + (uint32_t)kv * KV_BYTES +
+                                 (uint32_t)ch * (T * 128) + (uint32_t)(box * bt) * 128;
+            tma_load_3d(dst, kv ? (const void *)&tm.v : (const void *)&tm.k, ch * 64, seg.h, row,
+                        bar_addr(smem, D, B_FULL(s)));
+          }
         }
         ++it;
         // Find the next segment once this one's first stage is on its way
@@ -721,12 +724,12 @@ __device__ __forceinline__ bool arrive_and_check_last(const DecodeArgs &a, int u
 // LSE = ln sum_i exp(lse_i) and O = sum_i exp(lse_i - LSE) O_i, in one pass
 // with a running maximum per row.  The pieces are the tail slot of the
 // first CTA and the head slots of the following ones.  Every lane owns
-// D / 32 output columns; the loads of a batch of 4 pieces x 4 rows are
+// D / 32 output columns; the loads of a batch of 4 pieces x 2 rows are
 // independent, so a batch costs one memory round trip.
 template <int D, bool kBf16>
 __device__ void merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int rows, int unit, int lane) {
   constexpr int VEC = D / 32;
-  constexpr int PB = 4, RB = 4;  // pieces and rows per batch
+  constexpr int PB = 4, RB = 2;  // pieces and rows per batch
   const int n = sg.n_pieces, cf = sg.c_first;
   auto slot_of = [&](int i) -> size_t { return i == 0 ? (size_t)cf * 2 + 1 : (size_t)(cf + i) * 2; };
   const int col = lane * VEC;

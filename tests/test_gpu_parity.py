@@ -136,7 +136,7 @@ def test_edge_lengths(D, dtype, num_splits):
 @pytest.mark.parametrize("D", [64, 128])
 def test_page_sizes(page, D):
     if page == 192 and D == 64:
-        pytest.skip("192 neither divides nor is a multiple of the 128-key stage")
+        pytest.skip("192 neither divides nor is a multiple of the 128-key stage of D = 64")
     inp = make_inputs(wl(page_size=page, D=D, lengths="list:1,100,700,1030,2049", B=5, seed=page + D))
     for s in (0, 2):
         out, lse, _ = run_gpu(inp, num_splits=s)

@@ -94,6 +94,7 @@ def params(**kw):
 def test_plan_long_context_split():
     plan = mxa.mxa_plan(params(), 0, sm_count=148)
     assert plan.schedule == MXA_SCHED_BALANCED
+    # 16 tiles on 296 slots (two CTAs per SM): eff(16) = 256/296 = 0.865 is the first >= 0.85
     assert plan.units == 16 and plan.num_splits == 16 and plan.grid == 256
     assert plan.ctas_per_sm == 2 and plan.block_tokens == 64
     assert plan.needs_combine == 1 and plan.workspace_bytes > 0
