@@ -136,21 +136,31 @@ mxa_status_t mxa_plan(const mxa_decode_params_t *p, int num_splits, int sm_count
     out.grid = (int)(units * num_splits);
   } else {
     const int slots = sm_count * ctas_per_sm(p->D);
-    const int n_blocks_128 = (int)ceil_div_ll(p->max_seqlen_k, 128);
-    int max_splits = (int)ceil_div_ll(p->max_seqlen_k, T);
-    if (max_splits > 128) max_splits = 128;
-    if (max_splits < 1) max_splits = 1;
-    const double kv_head_bytes = (double)p->max_seqlen_k * p->D * 2.0 * 2.0;
-    int s = units > 0 ? mxa_num_splits_heuristic((int)units, sm_count, slots, n_blocks_128, max_splits,
-                                                 0, RT, kv_head_bytes)
-                      : 1;
-    if (s < 1) s = 1;
-    out.num_splits = s;
+    const long long max_blocks = ceil_div_ll(p->max_seqlen_k, T);
     if (p->B <= kMaxBalancedRows) {
+      // Balanced: every CTA streams the same number of KV blocks, so the
+      // wave efficiency n_waves / ceil(n_waves) of the num_splits rule is
+      // highest (1.0) for exactly one full wave of resident CTAs.  Units are
+      // not cut into pieces of fewer than 4 blocks on average (the rule's
+      // "no split below 4 blocks" floor), so tiny problems stay whole.
+      long long cap = units * (max_blocks + 3) / 4;
+      if (cap < 1) cap = 1;
       out.schedule = MXA_SCHED_BALANCED;
-      out.grid = (int)(units * s > 0 ? units * s : 1);
+      out.grid = (int)(slots < cap ? slots : cap);
+      out.num_splits = units > 0 ? (int)ceil_div_ll(out.grid, units) : 1;
     } else {
+      // Too many rows for the balanced prologue: the page's num_splits rule
+      // with the uniform schedule.
+      const int n_blocks_128 = (int)ceil_div_ll(p->max_seqlen_k, 128);
+      int max_splits = (int)(max_blocks > 128 ? 128 : max_blocks);
+      if (max_splits < 1) max_splits = 1;
+      const double kv_head_bytes = (double)p->max_seqlen_k * p->D * 2.0 * 2.0;
+      int s = mxa_num_splits_heuristic((int)units, sm_count, slots, n_blocks_128, max_splits, 0, RT,
+                                       kv_head_bytes);
+      if (s < 1) s = 1;
+      if (units * s > INT32_MAX) return MXA_ERR_UNSUPPORTED;
       out.schedule = MXA_SCHED_UNIFORM;
+      out.num_splits = s;
       out.grid = (int)(units * s);
     }
   }

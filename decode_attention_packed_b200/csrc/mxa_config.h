@@ -51,15 +51,25 @@ struct JobSlot {
   float ml[kMathWarps][kRowsPerTile][2];
 };
 
-constexpr size_t kBarrierBytes = 128;   // full[S], empty[S], qfull, qempty, job_full[J], job_empty[J]
-constexpr int kNumBarriers = 2 * kStages + 2 + 2 * kJobs;
+constexpr size_t kBarrierBytes = 128;   // full[S], empty[S], qfull, qempty, job_full[J], job_empty[J], merge
+constexpr int kNumBarriers = 2 * kStages + 2 + 2 * kJobs + 1;
 
 // Offsets inside the dynamic shared memory (base aligned to 1024 bytes).
 constexpr size_t smem_ring_off() { return 0; }
 constexpr size_t smem_q_off(int D) { return smem_ring_off() + kStages * stage_bytes(D); }
 constexpr size_t smem_desc_off(int D) { return smem_q_off(D) + q_tile_bytes(D); }
 constexpr size_t smem_jobs_off(int D) { return smem_desc_off(D) + sizeof(SegmentDesc); }
-constexpr size_t smem_bar_off(int D) { return smem_jobs_off(D) + kJobs * sizeof(JobSlot); }
+// The epilogue warp's staging buffer, used in turn for the rows of a job's
+// output before their bulk (TMA) stores (up to 16 rows x D fp32), and as the
+// landing zone of the pieces of a split unit being merged (partial rows
+// first, then the 16 LSE values of each piece).
+constexpr size_t kLandRows = 8 * 1024;
+constexpr size_t kLandBytes = kLandRows + 16 * kRowsPerTile * 4;
+constexpr size_t out_stage_bytes(int D) {
+  return (size_t)kRowsPerTile * D * 4 > kLandBytes ? (size_t)kRowsPerTile * D * 4 : kLandBytes;
+}
+constexpr size_t smem_out_off(int D) { return smem_jobs_off(D) + kJobs * sizeof(JobSlot); }
+constexpr size_t smem_bar_off(int D) { return smem_out_off(D) + out_stage_bytes(D); }
 constexpr size_t smem_total(int D) { return smem_bar_off(D) + kBarrierBytes; }
 
 constexpr int ctas_per_sm(int D) {

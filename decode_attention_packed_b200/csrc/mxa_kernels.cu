@@ -56,6 +56,7 @@ constexpr int B_QFULL = 2 * kStages;
 constexpr int B_QEMPTY = 2 * kStages + 1;
 constexpr int B_JOBFULL(int j) { return 2 * kStages + 2 + j; }
 constexpr int B_JOBEMPTY(int j) { return 2 * kStages + 2 + kJobs + j; }
+constexpr int B_MERGE = 2 * kStages + 2 + 2 * kJobs;  // pieces of a split unit landed by bulk loads
 
 // ---------------------------------------------------------------------------
 // Producer warp
@@ -264,6 +265,9 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
     prefetch_tmap(&tm.k);
     prefetch_tmap(&tm.v);
   }
+  // Inputs may be written by the kernel this launch depends on: read them
+  // only once that grid has completed and its writes are visible.
+  grid_dependency_wait();
   Cursor tail;
   bool has_tail;
   Cursor cur = cursor_start<D>(a, smem, lane, tail, has_tail);
@@ -680,6 +684,35 @@ __device__ __forceinline__ void store_out_vec(const DecodeArgs &a, int b, int t,
   }
 }
 
+// D / 32 consecutive values of packed row `rr`, rounded to the output type,
+// into the staging rows (row pitch D * 2 bytes).
+template <int D, bool kBf16>
+__device__ __forceinline__ void stage_out_vec(uint32_t stage, int rr, int col, const float *v) {
+  const uint32_t addr = stage + (uint32_t)(rr * D + col) * 2;
+  if constexpr (D / 32 == 4) {
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(pack2<kBf16>(v[0], v[1])),
+                 "r"(pack2<kBf16>(v[2], v[3])) : "memory");
+  } else {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(pack2<kBf16>(v[0], v[1])) : "memory");
+  }
+}
+
+// Bulk stores of `rows` staged output rows of a unit: the rows of one query
+// position t are the consecutive heads h * G + g and so one contiguous run
+// of out[b, t, :, :].  Issued by the calling lane.
+template <int D>
+__device__ __forceinline__ void store_out_rows(const DecodeArgs &a, int b, int h, int rt, int rows,
+                                               uint32_t stage) {
+  int r = 0;
+  while (r < rows) {
+    const int m = rt * kRowsPerTile + r, t = m / a.G, g = m % a.G;
+    const int r_end = min(rows, (t + 1) * a.G - rt * kRowsPerTile);
+    uint16_t *dst = reinterpret_cast<uint16_t *>(a.out) + ((size_t)(b * a.q_len + t) * a.Hq + (size_t)h * a.G + g) * D;
+    bulk_store(dst, stage + (uint32_t)(r * D * 2), (uint32_t)((r_end - r) * D * 2));
+    r = r_end;
+  }
+}
+
 // Output of a unit whose row sees no key at all (L_b = 0): O = 0, LSE = -inf.
 template <int D>
 __device__ void write_empty_unit(const DecodeArgs &a, int unit, int lane) {
@@ -720,58 +753,89 @@ __device__ __forceinline__ bool arrive_and_check_last(const DecodeArgs &a, int u
   }
 }
 
+// Room for partial rows in a landing zone that is a whole ring stage; its
+// LSEs follow.
+template <int D>
+constexpr uint32_t stage_land_rows() { return (uint32_t)stage_bytes(D) - 16 * kRowsPerTile * 4; }
+
 // Merge the n pieces of a split unit with the log-sum-exp identity,
 // LSE = ln sum_i exp(lse_i) and O = sum_i exp(lse_i - LSE) O_i, in one pass
 // with a running maximum per row.  The pieces are the tail slot of the
-// first CTA and the head slots of the following ones.  Every lane owns
-// D / 32 output columns; the loads of a batch of 4 pieces x 2 rows are
-// independent, so a batch costs one memory round trip.
+// first CTA and the head slots of the following ones.  Their partial rows
+// and LSEs are brought into a landing zone (`land`, with `land_rows` bytes
+// for rows and the LSEs after them) with bulk loads, up to 16 pieces at a
+// time, and merged from shared memory.  Every lane owns D / 32 output
+// columns.  Returns false if a bounded wait ran out.
 template <int D, bool kBf16>
-__device__ void merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int rows, int unit, int lane) {
+__device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int rows, int unit, int lane,
+                             uint32_t ostage, uint32_t land, uint32_t land_rows, uint32_t mbar,
+                             uint32_t &mk) {
   constexpr int VEC = D / 32;
-  constexpr int PB = 4, RB = 2;  // pieces and rows per batch
+  constexpr int RG = 8;  // rows merged per pass
+  const uint32_t kLandO = land_rows;
   const int n = sg.n_pieces, cf = sg.c_first;
   auto slot_of = [&](int i) -> size_t { return i == 0 ? (size_t)cf * 2 + 1 : (size_t)(cf + i) * 2; };
+  const uint32_t pbytes = (uint32_t)rows * D * 4;
+  const int cap = min(16, (int)(kLandO / pbytes));
+  const bool single = n <= cap;  // one landing serves every row group
   const int col = lane * VEC;
-  for (int r0 = 0; r0 < rows; r0 += RB) {
-    float m[RB], ssum[RB], acc[RB][VEC];
+  for (int r0 = 0; r0 < rows; r0 += RG) {
+    float m[RG], ssum[RG], acc[RG][VEC];
 #pragma unroll
-    for (int q = 0; q < RB; ++q) {
+    for (int q = 0; q < RG; ++q) {
       m[q] = -INFINITY;
       ssum[q] = 0.f;
 #pragma unroll
       for (int v = 0; v < VEC; ++v) acc[q][v] = 0.f;
     }
-    for (int i0 = 0; i0 < n; i0 += PB) {
-      float l[PB][RB], o[PB][RB][VEC];
-#pragma unroll
-      for (int p = 0; p < PB; ++p) {
-#pragma unroll
-        for (int q = 0; q < RB; ++q) {
-          const bool live = i0 + p < n && r0 + q < rows;
-          const size_t base = live ? slot_of(i0 + p) * kRowsPerTile + r0 + q : 0;
-          l[p][q] = live ? __ldcg(a.lse_part + base) : -INFINITY;
-#pragma unroll
-          for (int v = 0; v < VEC; ++v) o[p][q][v] = live ? __ldcg(a.o_part + base * D + col + v) : 0.f;
+    for (int i0 = 0; i0 < n; i0 += cap) {
+      const int k = min(cap, n - i0);
+      if (single && r0 > 0) goto landed;
+      fence_proxy_async_smem();  // earlier reads of the landing zone precede the new loads
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(mbar, (uint32_t)k * (pbytes + kRowsPerTile * 4));
+        for (int p = 0; p < k; ++p) {
+          const size_t sl = slot_of(i0 + p);
+          bulk_load(land + (uint32_t)p * pbytes, a.o_part + sl * kRowsPerTile * D, pbytes, mbar);
+          bulk_load(land + kLandO + (uint32_t)p * kRowsPerTile * 4, a.lse_part + sl * kRowsPerTile,
+                    kRowsPerTile * 4, mbar);
         }
       }
+      __syncwarp();
+      {
+        const bool ok = warp_wait_bounded(mbar, mk & 1, &g_mxa_err, kErrWaitFull, lane);
+        ++mk;
+        if (!ok) return false;
+      }
+    landed:
+      for (int p = 0; p < k; ++p) {
 #pragma unroll
-      for (int p = 0; p < PB; ++p) {
-#pragma unroll
-        for (int q = 0; q < RB; ++q) {
-          if (l[p][q] == -INFINITY) continue;  // an empty piece carries no weight
-          const float mn = fmaxf(m[q], l[p][q]);
+        for (int q = 0; q < RG; ++q) {
+          const int rr = r0 + q;
+          if (rr >= rows) break;
+          float l;
+          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l) : "r"(land + kLandO + (uint32_t)(p * kRowsPerTile + rr) * 4) : "memory");
+          if (l == -INFINITY) continue;  // an empty piece carries no weight
+          float o[VEC];
+          const uint32_t src = land + (uint32_t)p * pbytes + (uint32_t)(rr * D + col) * 4;
+          if constexpr (VEC == 4) {
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(o[0]), "=f"(o[1]), "=f"(o[2]), "=f"(o[3]) : "r"(src) : "memory");
+          } else {
+            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(o[0]), "=f"(o[1]) : "r"(src) : "memory");
+          }
+          const float mn = fmaxf(m[q], l);
           const float keep = m[q] == -INFINITY ? 0.f : expf(m[q] - mn);
-          const float w = expf(l[p][q] - mn);
+          const float w = expf(l - mn);
           ssum[q] = ssum[q] * keep + w;
 #pragma unroll
-          for (int v = 0; v < VEC; ++v) acc[q][v] = acc[q][v] * keep + w * o[p][q][v];
+          for (int v = 0; v < VEC; ++v) acc[q][v] = acc[q][v] * keep + w * o[v];
           m[q] = mn;
         }
       }
     }
 #pragma unroll
-    for (int q = 0; q < RB; ++q) {
+    for (int q = 0; q < RG; ++q) {
       const int rr = r0 + q;
       if (rr < rows) {
         const float inv = ssum[q] > 0.f ? 1.f / ssum[q] : 0.f;
@@ -780,12 +844,19 @@ __device__ void merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
         for (int v = 0; v < VEC; ++v) out_v[v] = acc[q][v] * inv;
         const float lse = m[q] == -INFINITY ? -INFINITY : m[q] + logf(ssum[q]);
         const int mrow = sg.rt * kRowsPerTile + rr, t = mrow / a.G, g = mrow % a.G, hq = sg.h * a.G + g;
-        store_out_vec<D, kBf16>(a, sg.b, t, hq, col, out_v);
+        stage_out_vec<D, kBf16>(ostage, rr, col, out_v);
         if (lane == 0 && a.lse != nullptr) a.lse[((size_t)sg.b * a.Hq + hq) * a.q_len + t] = lse;
       }
     }
   }
-  if (lane == 0) a.counters[unit] = 0ull;  // every piece has arrived; leave it clean
+  fence_proxy_async_smem();  // staged rows are read by the bulk stores
+  __syncwarp();
+  if (lane == 0) {
+    store_out_rows<D>(a, sg.b, sg.h, sg.rt, rows, ostage);
+    bulk_commit();
+    a.counters[unit] = 0ull;  // every piece has arrived; leave it clean
+  }
+  return true;
 }
 
 template <int D, bool kBf16>
@@ -798,6 +869,10 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
   JobSlot *jobs = reinterpret_cast<JobSlot *>(smem + smem_jobs_off(D));
   const int HR = a.Hkv * a.RT;
 
+  // Outputs and the workspace may still be in use by the kernel this launch
+  // depends on (an earlier call on the same buffers).
+  grid_dependency_wait();
+
   // Units of rows with L_b = 0 hold no KV block; one CTA per unit writes
   // their empty result.
   if (a.schedule == MXA_SCHED_BALANCED) {
@@ -809,13 +884,28 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
   }
 
   const int col = lane * VEC;
+  const uint32_t ostage = smem_addr(smem + smem_out_off(D));
+  const uint32_t oland = ostage;  // free again once this job's own rows have been stored
+  const uint32_t merge_bar = bar_addr(smem, D, B_MERGE);
+  uint32_t mk = 0;  // phases of the merge barrier used so far
   for (int jn = 0;; ++jn) {
     const int j = jn % kJobs, jk = jn / kJobs;
-    if (!warp_wait_bounded(bar_addr(smem, D, B_JOBFULL(j)), jk & 1, &g_mxa_err, kErrWaitFull, lane)) return;
+    // Leaving: bulk stores this warp issued must be done with shared memory
+    // (and complete) before the CTA exits.
+    if (!warp_wait_bounded(bar_addr(smem, D, B_JOBFULL(j)), jk & 1, &g_mxa_err, kErrWaitFull, lane)) {
+      if (lane == 0) bulk_wait_all();
+      return;
+    }
     const SegmentDesc sg = jobs[j].seg;
-    if (sg.kind < 0) return;
+    if (sg.kind < 0) {
+      if (lane == 0) bulk_wait_all();
+      return;
+    }
     const int stage = jobs[j].stage;
     const uint32_t sbase = ring + (uint32_t)stage * (2 * KV_BYTES);
+    // the staging rows are free once earlier bulk stores have read them
+    if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
     const int rows = min(kRowsPerTile, a.M - sg.rt * kRowsPerTile);
     const int unit = (sg.b * a.Hkv + sg.h) * a.RT + sg.rt;
     const int slot = sg.kind - 1;  // partial slot (kind 1 -> head slot 0, kind 2 -> tail slot 1)
@@ -867,35 +957,71 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
           }
         }
       }
-      const float lse = __shfl_sync(0xffffffffu, my_lse, rr);
-      const int m = sg.rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G, hq = sg.h * a.G + g;
       if (sg.kind == 0) {
-        store_out_vec<D, kBf16>(a, sg.b, t, hq, col, acc);
-        if (lane == 0 && a.lse != nullptr) a.lse[((size_t)sg.b * a.Hq + hq) * a.q_len + t] = lse;
-      } else {
-        float *dst = a.o_part + (((size_t)blockIdx.x * 2 + slot) * kRowsPerTile + rr) * D + col;
+        stage_out_vec<D, kBf16>(ostage, rr, col, acc);
+      } else {  // fp32 partial rows, pitch D * 4 bytes
+        const uint32_t addr = ostage + (uint32_t)(rr * D + col) * 4;
         if constexpr (VEC == 4) {
-          *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(acc[0]), "f"(acc[1]),
+                       "f"(acc[2]), "f"(acc[3]) : "memory");
         } else {
-          *reinterpret_cast<float2 *>(dst) = make_float2(acc[0], acc[1]);
+          asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(acc[0]), "f"(acc[1]) : "memory");
         }
-        if (lane == 0) a.lse_part[((size_t)blockIdx.x * 2 + slot) * kRowsPerTile + rr] = lse;
+      }
+    }
+    // row statistics: lane r < rows owns row r
+    if (lane < rows) {
+      if (sg.kind == 0) {
+        const int m = sg.rt * kRowsPerTile + lane, t = m / a.G, g = m % a.G, hq = sg.h * a.G + g;
+        if (a.lse != nullptr) a.lse[((size_t)sg.b * a.Hq + hq) * a.q_len + t] = my_lse;
+      } else {
+        a.lse_part[((size_t)blockIdx.x * 2 + slot) * kRowsPerTile + lane] = my_lse;
       }
     }
     // Give the stage back to the producer and the hand-off slot to the math
     // warps.  This warp only read the stage; the math warps fenced their
-    // generic writes to it before handing it over.
+    // generic writes to it before handing it over.  Then write the staged
+    // rows out with bulk stores.
+    fence_proxy_async_smem();  // staged rows are read by the bulk stores
     __syncwarp();
+    // A merge whose pieces all fit the landing buffer does not need the
+    // stage; otherwise the stage is kept as the landing zone until this
+    // piece has been counted (and merged, if it was the last).
+    const bool hold = sg.kind != 0 && (uint32_t)sg.n_pieces * rows * D * 4 > (uint32_t)kLandRows;
     if (lane == 0) {
-      mbar_arrive_cnt(bar_addr(smem, D, B_EMPTY(stage)), kMathWarps);
       mbar_arrive(bar_addr(smem, D, B_JOBEMPTY(j)));
+      if (!hold) mbar_arrive_cnt(bar_addr(smem, D, B_EMPTY(stage)), kMathWarps);
+      if (sg.kind == 0) {
+        store_out_rows<D>(a, sg.b, sg.h, sg.rt, rows, ostage);
+      } else {
+        bulk_store(a.o_part + ((size_t)blockIdx.x * 2 + slot) * kRowsPerTile * D, ostage, (uint32_t)(rows * D * 4));
+      }
+      bulk_commit();
     }
-    if (sg.kind != 0) {  // a piece of a split unit: the last piece to arrive merges them all
+    if (sg.kind != 0) {
+      // A piece of a split unit: the last piece to arrive merges them all.
+      if (lane == 0) {
+        bulk_wait_all();  // this piece's partial rows are in global memory
+        bulk_wait_read_all();
+      }
       __threadfence();
       __syncwarp();
+      bool ok = true;
       if (arrive_and_check_last(a, unit, sg.n_pieces, lane)) {
         __threadfence();
-        merge_pieces<D, kBf16>(a, sg, rows, unit, lane);
+        ok = hold ? merge_pieces<D, kBf16>(a, sg, rows, unit, lane, ostage, sbase, stage_land_rows<D>(),
+                                           merge_bar, mk)
+                  : merge_pieces<D, kBf16>(a, sg, rows, unit, lane, ostage, oland, (uint32_t)kLandRows,
+                                           merge_bar, mk);
+      }
+      if (hold) {
+        fence_proxy_async_smem();  // reads of the landing zone precede the stage's next TMA loads
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cnt(bar_addr(smem, D, B_EMPTY(stage)), kMathWarps);
+      }
+      if (!ok) {
+        if (lane == 0) bulk_wait_all();
+        return;
       }
     }
   }
@@ -924,9 +1050,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(bar_addr(smem, D, B_JOBFULL(j)), kMathWarps);
       mbar_init(bar_addr(smem, D, B_JOBEMPTY(j)), 1);
     }
+    mbar_init(bar_addr(smem, D, B_MERGE), 1);
     fence_mbar_init();
   }
   __syncthreads();
+  // A dependent launch (the next call on this stream) may start its CTAs as
+  // SM slots free up; it reads and writes global memory only after this
+  // grid has completed (grid_dependency_wait in its producer and epilogue
+  // warps).  The math warps touch shared memory only.
+  grid_launch_dependents();
   if (warp == kProducerWarp) {
     producer_warp<D, kBf16>(tm, a, smem, lane);
   } else if (warp == kEpilogueWarp) {
@@ -1094,7 +1226,17 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
       !encode_kv_map(&tm.v, L.v_cache, D, p.Hkv, pool_tokens, a.box_tokens, kBf16))
     return MXA_ERR_CUDA;
 
-  mxa_split_kernel<D, kBf16><<<plan.grid, kThreads, smem_total(D), stream>>>(tm, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)plan.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem_total(D);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, mxa_split_kernel<D, kBf16>, tm, a) != cudaSuccess) return MXA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? MXA_OK : MXA_ERR_CUDA;
 }
 

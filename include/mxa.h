@@ -140,8 +140,13 @@ MXA_API int mxa_num_splits_heuristic(int tiles, int sm_count, int slots, int num
 
 /* Resolve a plan for `params`.
  *   num_splits > 0 : UNIFORM schedule with that many splits per unit.
- *   num_splits == 0: automatic: s from mxa_num_splits_heuristic, BALANCED
- *                    schedule with grid = units * s.
+ *   num_splits == 0: automatic: BALANCED schedule over one full wave of
+ *                    resident CTAs (grid = SMs x CTAs per SM, the wave
+ *                    efficiency optimum when every CTA carries the same
+ *                    work), capped at units * ceil(blocks per unit / 4) so
+ *                    no unit is cut into pieces under 4 blocks on average;
+ *                    for B above 16384 rows, UNIFORM with s from
+ *                    mxa_num_splits_heuristic.
  *   sm_count > 0   : plan for that many SMs (pure host computation);
  *   sm_count <= 0  : query the current CUDA device (MXA_ERR_CUDA without one).
  * Errors: MXA_ERR_INVALID_ARG for a NULL pointer or an inconsistent shape

@@ -94,10 +94,20 @@ def params(**kw):
 def test_plan_long_context_split():
     plan = mxa.mxa_plan(params(), 0, sm_count=148)
     assert plan.schedule == MXA_SCHED_BALANCED
-    # 16 tiles on 296 slots (two CTAs per SM): eff(16) = 256/296 = 0.865 is the first >= 0.85
-    assert plan.units == 16 and plan.num_splits == 16 and plan.grid == 256
+    # one full wave of two CTAs per SM over 16 units of 256 blocks
+    assert plan.units == 16 and plan.grid == 296 and plan.num_splits == 19
     assert plan.ctas_per_sm == 2 and plan.block_tokens == 64
     assert plan.needs_combine == 1 and plan.workspace_bytes > 0
+
+
+def test_plan_does_not_split_tiny_problems():
+    # one unit of 4 blocks: pieces would be under 4 blocks, so one CTA
+    p = params(B=1, Hq=4, Hkv=1, D=64, max_seqlen_k=512, max_pages_per_seq=8, num_pages=8)
+    plan = mxa.mxa_plan(p, 0, sm_count=148)
+    assert plan.grid == 1 and plan.needs_combine == 0 and plan.workspace_bytes == 0
+    # 1024 units of up to 256 blocks: capped by the wave
+    p = params(B=128, Hq=16, Hkv=8, D=64, max_seqlen_k=16384, max_pages_per_seq=1024, num_pages=20000)
+    assert mxa.mxa_plan(p, 0, sm_count=148).grid == 296
 
 
 def test_plan_uniform_and_row_tiles():
