@@ -3,7 +3,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mxa|reference]
                     [--workload gqa_decode] [--num-splits S]
 
-One step = one decode call (split kernel + merge) over the whole workload:
+One step = one decode call (one launch of the split kernel, which also merges
+units split across CTAs) over the whole workload:
 B = 32 rows, Hq = 32, Hkv = 8, head_dim 128, bf16, pages of 16 slots in a
 seeded random permutation, KV lengths uniform in [1, 4096].  Inputs are
 seeded synthetic data.  KV pools rotate over three copies (each larger than
@@ -33,6 +34,12 @@ import torch  # noqa: E402
 from decode_attention_packed_b200.workloads import WORKLOADS, make_inputs, workload  # noqa: E402
 
 METRIC = "decode-attn µs/call and KV-read GB/s as % of B200 HBM peak (1 GPU)"
+
+# DRAM bytes (read + written) per launch of the split kernel on the default
+# workload, from an ncu capture (profiles/mxa_split_kernel_gqa_decode.md),
+# keyed by a hash of the kernel sources it was taken on: once the kernel
+# changes the number no longer applies and the bench reports null.
+MEASURED_TRAFFIC = {"3f7b4c77cd120044": 249441792}
 DEFAULT_WORKLOAD = "gqa_decode"
 FALLBACK_HBM_GBS = 6650.0
 N_POOLS = 3
@@ -59,6 +66,20 @@ def measured_peak():
         except Exception:
             pass
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    import glob
+    import hashlib
+    csrc = os.path.join(ROOT, "decode_attention_packed_b200", "csrc")
+    files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")) +
+                   glob.glob(os.path.join(csrc, "*.h")))
+    h = hashlib.sha256()
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def algorithmic_bytes(inp) -> dict:
@@ -236,7 +257,7 @@ def main():
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=dev)
     nbytes = algorithmic_bytes(inp)
-    launches_per_call = 1 + prep.plan.needs_combine
+    launches_per_call = 1  # the split kernel merges split units itself
 
     def call(i):
         k, v = pools[i % N_POOLS]
@@ -337,10 +358,11 @@ def main():
                    "l2": f"KV rotates over {N_POOLS} device copies of {nbytes['kv'] / 1e6:.0f} MB (> L2)",
                    "parallelism": f"dp{world} (independent decode rows per rank)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4),
+                     "traffic": MEASURED_TRAFFIC.get(kernel_source_hash()) if w.name == DEFAULT_WORKLOAD else None,
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                      else "fallback 6.65 TB/s",
-                     "kernel": "mxa_split_kernel (+ merge; per-call time)"},
+                     "kernel": "mxa_split_kernel (one launch per call; split units merged inside)"},
         "e2e": {"value": round(nbytes["kv"] * world / (e2e_s / e2e_steps) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": args.steps * launches_per_call,
