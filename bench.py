@@ -82,6 +82,15 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def workload_config(w, nbytes: dict, world: int) -> dict:
+    """The `config` object of the JSON line; both arms report the same one."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "q_len": w.q_len,
+            "page_size": w.page_size, "lengths": w.lengths, "causal": w.causal,
+            "kv_dtype": w.dtype, "kv_bytes_per_call": nbytes["kv"],
+            "l2": f"KV rotates over {N_POOLS} device copies of {nbytes['kv'] / 1e6:.0f} MB (> L2)",
+            "parallelism": f"dp{world} (independent decode rows per rank)"}
+
+
 def algorithmic_bytes(inp) -> dict:
     """Bytes one decode call must move at minimum (read KV, Q, block table,
     lengths; write O and LSE)."""
@@ -223,8 +232,7 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(tot_t / args.steps * 1e3, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                   "q_len": w.q_len, "page_size": w.page_size, "kv_dtype": w.dtype},
+        "config": workload_config(w, algorithmic_bytes(inp), world),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": omp_threads(),
                          "kind": "oracle", "sample": f"first {rows} of {w.B} rows per step"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -352,11 +360,8 @@ def main():
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "q_len": w.q_len,
-                   "page_size": w.page_size, "lengths": w.lengths, "causal": w.causal,
-                   "kv_bytes_per_call": nbytes["kv"], "plan": prep.plan.as_dict(),
-                   "l2": f"KV rotates over {N_POOLS} device copies of {nbytes['kv'] / 1e6:.0f} MB (> L2)",
-                   "parallelism": f"dp{world} (independent decode rows per rank)"},
+        "config": workload_config(w, nbytes, world),
+        "plan": prep.plan.as_dict(),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "traffic": MEASURED_TRAFFIC.get(kernel_source_hash()) if w.name == DEFAULT_WORKLOAD else None,
