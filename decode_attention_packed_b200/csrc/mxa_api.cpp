@@ -146,6 +146,7 @@ mxa_status_t mxa_plan(const mxa_decode_params_t *p, int num_splits, int sm_count
       long long cap = units * (max_blocks + 3) / 4;
       if (cap < 1) cap = 1;
       out.schedule = MXA_SCHED_BALANCED;
+      out.unit_cost = kUnitCost;
       out.grid = (int)(slots < cap ? slots : cap);
       out.num_splits = units > 0 ? (int)ceil_div_ll(out.grid, units) : 1;
     } else {
@@ -177,6 +178,7 @@ mxa_status_t mxa_plan_balanced(const mxa_decode_params_t *p, int grid, int sm_co
   if (st != MXA_OK) return st;
   if (p->B > kMaxBalancedRows) return MXA_ERR_UNSUPPORTED;
   out.schedule = MXA_SCHED_BALANCED;
+  out.unit_cost = kUnitCost;
   out.grid = grid;
   out.num_splits = out.units > 0 ? (grid + out.units - 1) / out.units : 1;
   finish_plan(p, &out);
@@ -206,6 +208,9 @@ mxa_status_t mxa_decode_fwd_with_plan(const void *q, const void *k_cache, const 
   mxa_plan_t use = *plan;
   if (use.schedule != MXA_SCHED_UNIFORM && use.schedule != MXA_SCHED_BALANCED) return MXA_ERR_INVALID_ARG;
   if (use.grid < 1 || use.num_splits < 1) return MXA_ERR_INVALID_ARG;
+  if (use.schedule == MXA_SCHED_BALANCED && (use.unit_cost < 0 || use.unit_cost > kMaxUnitCost))
+    return MXA_ERR_INVALID_ARG;
+  if (use.schedule == MXA_SCHED_UNIFORM) use.unit_cost = 0;
   finish_plan(p, &use);
   if (use.schedule == MXA_SCHED_UNIFORM && (long long)use.units * use.num_splits != use.grid)
     return MXA_ERR_INVALID_ARG;

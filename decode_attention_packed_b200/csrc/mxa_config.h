@@ -15,7 +15,9 @@ constexpr int kJobs = 2;                                // epilogue hand-off slo
 constexpr int kSmemPerSm = 228 * 1024;                  // B200 shared memory per SM
 constexpr int kSmemReservedPerCta = 1024;               // driver-reserved shared memory per CTA
 constexpr int kMaxThreadsPerSm = 2048;
-constexpr int kMaxBalancedRows = 16384;                 // balanced schedule scans B rows in smem
+constexpr int kMaxBalancedRows = 12288;                 // balanced schedule scans B rows in smem
+constexpr int kUnitCost = 2;                            // fixed cost of a unit, in KV blocks
+constexpr int kMaxUnitCost = 64;
 
 // KV tokens per pipeline stage: every stage carries T x D elements of K and
 // of V (16 KiB each in 16-bit types), so T = 8192 / D.  Three stages per CTA
@@ -94,6 +96,6 @@ static_assert(2 * (smem_total(128) + kSmemReservedPerCta) <= (size_t)kSmemPerSm,
               "D = 128 layout must leave room for two CTAs per SM");
 static_assert(2 * (smem_total(64) + kSmemReservedPerCta) <= (size_t)kSmemPerSm,
               "D = 64 layout must leave room for two CTAs per SM");
-static_assert((size_t)kMaxBalancedRows * 4 + 4 * 32 <= kStages * stage_bytes(64), "prologue scan fits the ring");
+static_assert((size_t)kMaxBalancedRows * 8 <= kStages * stage_bytes(64), "prologue scan fits the ring");
 
 }  // namespace mxa

@@ -62,13 +62,16 @@ constexpr int B_MERGE = 2 * kStages + 2 + 2 * kJobs;  // pieces of a split unit 
 // Producer warp
 // ---------------------------------------------------------------------------
 
-// Cursor over this CTA's range of KV blocks: (row b, KV-head x row-tile hr,
-// block blk), `remaining` blocks left.
+// Cursor over this CTA's range of work.  BALANCED: positions in a
+// flattened cost space in which every unit (batch row b with nb > 0 KV
+// blocks, KV head x row tile hr) spans unit_cost + nb positions: first its
+// fixed cost, then one position per KV block.  `x` is the position of block
+// `blk` of the current unit and `end` closes the CTA's range.  UNIFORM:
+// positions are the unit's block indices.
 struct Cursor {
   int b, hr, blk;
-  long long remaining;
-  long long x;        // flattened index of block blk (balanced schedule)
-  long long per_cta;  // blocks per CTA range (balanced schedule)
+  long long x, end;
+  long long per_cta;  // positions per CTA range (balanced schedule)
   int L, nb;          // length and blocks of row b
   int L_next;         // prefetched length of row b + 1
 };
@@ -82,13 +85,13 @@ __device__ __forceinline__ void cursor_enter_row(Cursor &c, const DecodeArgs &a,
 }
 
 // The segment at the cursor (a contiguous block range of one unit); the
-// cursor moves past it.
+// cursor moves past it, and past the fixed cost of the unit that follows.
 template <int D>
 __device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
   const int HR = a.Hkv * a.RT;
   SegmentDesc s;
-  const long long left = c.nb - c.blk;
-  const int len = (int)(left < c.remaining ? left : c.remaining);
+  const long long left = c.nb - c.blk, room = c.end - c.x;
+  const int len = (int)(left < room ? left : room);
   s.b = c.b;
   s.h = c.hr / a.RT;
   s.rt = c.hr % a.RT;
@@ -97,7 +100,7 @@ __device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
   s.L = c.L;
   s.kind = (s.blk_beg == 0 && s.blk_end == c.nb) ? 0 : (s.blk_beg > 0 ? 1 : 2);
   if (a.schedule == MXA_SCHED_BALANCED) {
-    const long long xs = c.x - c.blk;  // flattened index of the unit's first block
+    const long long xs = c.x - c.blk;  // position of the unit's first block
     s.c_first = (int)(xs / c.per_cta);
     s.n_pieces = (int)((xs + c.nb - 1) / c.per_cta) - s.c_first + 1;
   } else {
@@ -107,42 +110,43 @@ __device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
   }
   s.pad[0] = s.pad[1] = s.pad[2] = 0;
 
-  c.remaining -= len;
   c.x += len;
   c.blk += len;
   if (c.blk == c.nb) {
     c.blk = 0;
     if (++c.hr == HR) {
       c.hr = 0;
-      if (c.remaining > 0 && c.b + 1 < a.B) {
+      if (c.x + a.unit_cost < c.end && c.b + 1 < a.B) {
         ++c.b;
         cursor_enter_row<D>(c, a, clamp_len(c.L_next, a.max_seqlen_k));
-        while (c.nb == 0 && c.b + 1 < a.B) {  // rows without keys hold no blocks
+        while (c.nb == 0 && c.b + 1 < a.B) {  // rows without keys hold no units
           ++c.b;
           cursor_enter_row<D>(c, a, clamp_len(a.seqlens[c.b], a.max_seqlen_k));
         }
       } else {
-        c.remaining = 0;
+        c.end = c.x;
       }
     }
+    c.x += a.unit_cost;  // the next unit's first block follows its fixed cost
   }
   return s;
 }
 
-// This CTA's range of the flattened block space.  BALANCED: the blocks of
-// all units laid end to end (row-major over (b, KV head, row tile)) and cut
-// into gridDim.x equal ranges; the prefix sum over rows is built in the
-// (still unused) ring by this warp alone.  UNIFORM: block range
-// [si * chunk, (si + 1) * chunk) of unit blockIdx.x / splits.
+// This CTA's range of work.  BALANCED: the cost space of all units laid end
+// to end (row-major over (b, KV head, row tile)) is cut into gridDim.x equal
+// ranges; the prefix sum over rows, and the lengths themselves, are kept in
+// the (still unused) ring by this warp alone, so the rows a range starts
+// and ends in are known without another read of global memory.  UNIFORM: block range [si * chunk, (si + 1) * chunk) of
+// unit blockIdx.x / splits.
 template <int D>
 __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cursor &tail, bool &has_tail) {
   constexpr int T = block_tokens(D);
   const int HR = a.Hkv * a.RT;
+  const int V = a.unit_cost;
   Cursor c;
   c.hr = 0;
   c.blk = 0;
-  c.remaining = 0;
-  c.x = 0;
+  c.x = c.end = 0;
   c.per_cta = 1;
   c.L = c.nb = c.L_next = 0;
   has_tail = false;
@@ -155,18 +159,23 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
     c.nb = (c.L + T - 1) / T;
     const int beg = si * a.chunk_blocks, end = min(beg + a.chunk_blocks, c.nb);
     c.blk = beg;
-    c.remaining = end > beg ? end - beg : 0;
+    c.x = beg;
+    c.end = end > beg ? end : beg;
     c.L_next = 0;
     return c;
   }
-  int *scan = reinterpret_cast<int *>(smem + smem_ring_off());
+  int *scan = reinterpret_cast<int *>(smem + smem_ring_off());  // [B] prefix of unit positions
+  int *lens = scan + a.B;                                        // [B] lengths, clamped
   const int chunk = (a.B + 31) / 32;
   const int lo = min(lane * chunk, a.B), hi = min(lo + chunk, a.B);
   int sum = 0;
   for (int i = lo; i < hi; ++i) {
-    const int nb = (clamp_len(a.seqlens[i], a.max_seqlen_k) + T - 1) / T;
-    scan[i] = nb;
-    sum += nb;
+    const int L = clamp_len(a.seqlens[i], a.max_seqlen_k);
+    lens[i] = L;
+    const int nb = (L + T - 1) / T;
+    const int w = nb > 0 ? nb + V : 0;  // positions of one unit of row i
+    scan[i] = w;
+    sum += w;
   }
   __syncwarp();
   int incl = sum;  // inclusive warp scan of the lane sums
@@ -179,7 +188,7 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
   int run = incl - sum;
   for (int i = lo; i < hi; ++i) {
     run += scan[i];
-    scan[i] = run;  // inclusive prefix of blocks per row
+    scan[i] = run;  // inclusive prefix of unit positions per row
   }
   __syncwarp();
   const long long NB = (long long)HR * total;
@@ -187,50 +196,55 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
   const long long x0 = (long long)blockIdx.x * c.per_cta;
   c.b = 0;
   if (x0 < NB) {
-    int lo_b = 0, hi_b = a.B - 1;  // first row whose blocks end past x0
+    const long long x1 = c.per_cta < NB - x0 ? x0 + c.per_cta : NB;
+    int lo_b = 0, hi_b = a.B - 1;  // first row whose positions end past x0
     while (lo_b < hi_b) {
       const int mid = (lo_b + hi_b) >> 1;
       if ((long long)HR * scan[mid] > x0) hi_b = mid; else lo_b = mid + 1;
     }
     const long long pre = lo_b > 0 ? scan[lo_b - 1] : 0;
-    const long long nb = scan[lo_b] - pre;
+    const long long w = scan[lo_b] - pre;  // > 0: the row holds position x0
     const long long off = x0 - (long long)HR * pre;
+    const long long pos = off % w;
     c.b = lo_b;
-    c.hr = (int)(off / nb);
-    c.blk = (int)(off % nb);
-    c.remaining = c.per_cta < NB - x0 ? c.per_cta : NB - x0;
-    c.x = x0;
-    c.nb = (int)nb;  // from the scan: the length itself is first needed later
-    c.L = clamp_len(a.seqlens[c.b], a.max_seqlen_k);
-    c.L_next = c.b + 1 < a.B ? a.seqlens[c.b + 1] : 0;
+    c.hr = (int)(off / w);
+    c.nb = (int)(w - V);  // from the scan: the length itself is first needed later
+    c.blk = pos > V ? (int)(pos - V) : 0;
+    c.x = x0 - pos + V + c.blk;
+    c.end = x1;
+    c.L = lens[c.b];
+    c.L_next = c.b + 1 < a.B ? lens[c.b + 1] : 0;
 
     // If the range ends inside a unit that starts within it (a tail piece),
     // that piece is handled first: its other pieces are then also done early
     // in their CTAs, and the unit's merge overlaps streaming instead of
     // lengthening the end of the kernel.
-    const long long xl = x0 + c.remaining - 1;
+    const long long xl = x1 - 1;
     int lb = lo_b, hb = a.B - 1;
     while (lb < hb) {
       const int mid = (lb + hb) >> 1;
       if ((long long)HR * scan[mid] > xl) hb = mid; else lb = mid + 1;
     }
     const long long pre_l = lb > 0 ? scan[lb - 1] : 0;
-    const long long nb_l = scan[lb] - pre_l;
+    const long long w_l = scan[lb] - pre_l;
     const long long off_l = xl - (long long)HR * pre_l;
-    const int hr_l = (int)(off_l / nb_l), blk_l = (int)(off_l % nb_l);
-    const long long x_t = xl - blk_l;  // flattened index of that unit's first block
-    if (blk_l + 1 < nb_l && x_t > x0) {
-      tail.b = lb;
-      tail.hr = hr_l;
-      tail.blk = 0;
-      tail.remaining = blk_l + 1;
-      tail.x = x_t;
-      tail.per_cta = c.per_cta;
-      tail.nb = (int)nb_l;
-      tail.L = clamp_len(a.seqlens[lb], a.max_seqlen_k);
-      tail.L_next = 0;
-      has_tail = true;
-      c.remaining = x_t - x0;
+    const long long pos_l = off_l % w_l;
+    if (pos_l >= V) {  // xl falls on a KV block of that unit
+      const int nb_l = (int)(w_l - V), blk_l = (int)(pos_l - V);
+      const long long x_t = xl - blk_l;  // position of that unit's first block
+      if (blk_l + 1 < nb_l && x_t - V > x0) {
+        tail.b = lb;
+        tail.hr = (int)(off_l / w_l);
+        tail.blk = 0;
+        tail.x = x_t;
+        tail.end = x1;
+        tail.per_cta = c.per_cta;
+        tail.nb = nb_l;
+        tail.L = lens[lb];
+        tail.L_next = 0;
+        has_tail = true;
+        c.end = x_t - V;  // the main walk stops where that unit begins
+      }
     }
   }
   __syncwarp();
@@ -271,7 +285,7 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
   Cursor tail;
   bool has_tail;
   Cursor cur = cursor_start<D>(a, smem, lane, tail, has_tail);
-  auto more = [&]() { return has_tail || (cur.remaining > 0 && cur.nb > 0); };
+  auto more = [&]() { return has_tail || (cur.x < cur.end && cur.nb > 0); };
   auto take = [&]() {
     if (has_tail) {
       has_tail = false;
@@ -685,15 +699,15 @@ __device__ __forceinline__ void store_out_vec(const DecodeArgs &a, int b, int t,
 }
 
 // D / 32 consecutive values of packed row `rr`, rounded to the output type,
-// into the staging rows (row pitch D * 2 bytes).
+// into the staging rows at shared address `stage` (row pitch D * 2 bytes).
+// A plain store, so the compiler may overlap it with the loads of other rows.
 template <int D, bool kBf16>
-__device__ __forceinline__ void stage_out_vec(uint32_t stage, int rr, int col, const float *v) {
-  const uint32_t addr = stage + (uint32_t)(rr * D + col) * 2;
+__device__ __forceinline__ void stage_out_vec(uint8_t *smem, uint32_t stage, int rr, int col, const float *v) {
+  uint8_t *dst = smem + (stage - smem_addr(smem)) + (rr * D + col) * 2;
   if constexpr (D / 32 == 4) {
-    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(pack2<kBf16>(v[0], v[1])),
-                 "r"(pack2<kBf16>(v[2], v[3])) : "memory");
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(pack2<kBf16>(v[0], v[1]), pack2<kBf16>(v[2], v[3]));
   } else {
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(pack2<kBf16>(v[0], v[1])) : "memory");
+    *reinterpret_cast<uint32_t *>(dst) = pack2<kBf16>(v[0], v[1]);
   }
 }
 
@@ -736,13 +750,14 @@ __device__ void write_empty_unit(const DecodeArgs &a, int unit, int lane) {
 // Count this piece of a split unit; true (in every lane) for the piece that
 // completes it.  The counter carries the call's epoch in its high half, so a
 // count left by an earlier (failed) call is not mistaken for this call's.
-// The retry loop runs on all lanes; only lane 0 touches memory.
-__device__ __forceinline__ bool arrive_and_check_last(const DecodeArgs &a, int unit, int n, int lane) {
+// `guess` is lane 0's earlier read of the counter: when no other piece has
+// arrived since, the first compare-and-swap succeeds.  The retry loop runs
+// on all lanes; only lane 0 touches memory.
+__device__ __forceinline__ bool arrive_and_check_last(const DecodeArgs &a, int unit, int n, int lane,
+                                                      unsigned long long guess) {
   unsigned long long *cnt = a.counters + unit;
   const unsigned long long ep = a.epoch;
-  unsigned long long cur = 0;
-  if (lane == 0) cur = atomicAdd(cnt, 0ull);
-  cur = __shfl_sync(0xffffffffu, cur, 0);
+  unsigned long long cur = __shfl_sync(0xffffffffu, guess, 0);
   for (;;) {
     const unsigned long long want = (cur >> 32) == ep ? cur + 1ull : ((ep << 32) | 1ull);
     unsigned long long prev = 0;
@@ -759,96 +774,119 @@ template <int D>
 constexpr uint32_t stage_land_rows() { return (uint32_t)stage_bytes(D) - 16 * kRowsPerTile * 4; }
 
 // Merge the n pieces of a split unit with the log-sum-exp identity,
-// LSE = ln sum_i exp(lse_i) and O = sum_i exp(lse_i - LSE) O_i, in one pass
-// with a running maximum per row.  The pieces are the tail slot of the
-// first CTA and the head slots of the following ones.  Their partial rows
-// and LSEs are brought into a landing zone (`land`, with `land_rows` bytes
-// for rows and the LSEs after them) with bulk loads, up to 16 pieces at a
-// time, and merged from shared memory.  Every lane owns D / 32 output
-// columns.  Returns false if a bounded wait ran out.
+// LSE = ln sum_i exp(lse_i) and O = sum_i exp(lse_i - LSE) O_i, in two
+// passes.  First the row statistics: the pieces' LSEs are read straight
+// from global memory, spread over a power-of-two group of lanes per row,
+// and reduced with a running maximum.  Then the weighted sum: the pieces'
+// partial rows and LSEs are brought into a landing zone (`land`, with
+// `land_rows` bytes for rows and the LSEs after them) with bulk loads, up
+// to 16 pieces at a time, and every lane accumulates its D / 32 columns of
+// every row.  With the weights known up front the products are independent
+// of one another, so the loads of many rows and pieces overlap.  The
+// pieces are the tail slot of the first CTA and the head slots of the
+// following ones.  Returns false if a bounded wait ran out.
 template <int D, bool kBf16>
 __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int rows, int unit, int lane,
-                             uint32_t ostage, uint32_t land, uint32_t land_rows, uint32_t mbar,
-                             uint32_t &mk) {
+                             uint8_t *smem, uint32_t ostage, uint32_t land, uint32_t land_rows,
+                             uint32_t mbar, uint32_t &mk) {
   constexpr int VEC = D / 32;
-  constexpr int RG = 8;  // rows merged per pass
-  const uint32_t kLandO = land_rows;
+  constexpr float kLog2e = 1.4426950408889634f;
   const int n = sg.n_pieces, cf = sg.c_first;
   auto slot_of = [&](int i) -> size_t { return i == 0 ? (size_t)cf * 2 + 1 : (size_t)(cf + i) * 2; };
+
   const uint32_t pbytes = (uint32_t)rows * D * 4;
-  const int cap = min(16, (int)(kLandO / pbytes));
-  const bool single = n <= cap;  // one landing serves every row group
-  const int col = lane * VEC;
-  for (int r0 = 0; r0 < rows; r0 += RG) {
-    float m[RG], ssum[RG], acc[RG][VEC];
-#pragma unroll
-    for (int q = 0; q < RG; ++q) {
-      m[q] = -INFINITY;
-      ssum[q] = 0.f;
-#pragma unroll
-      for (int v = 0; v < VEC; ++v) acc[q][v] = 0.f;
-    }
-    for (int i0 = 0; i0 < n; i0 += cap) {
-      const int k = min(cap, n - i0);
-      if (single && r0 > 0) goto landed;
-      fence_proxy_async_smem();  // earlier reads of the landing zone precede the new loads
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(mbar, (uint32_t)k * (pbytes + kRowsPerTile * 4));
-        for (int p = 0; p < k; ++p) {
-          const size_t sl = slot_of(i0 + p);
-          bulk_load(land + (uint32_t)p * pbytes, a.o_part + sl * kRowsPerTile * D, pbytes, mbar);
-          bulk_load(land + kLandO + (uint32_t)p * kRowsPerTile * 4, a.lse_part + sl * kRowsPerTile,
-                    kRowsPerTile * 4, mbar);
-        }
-      }
-      __syncwarp();
-      {
-        const bool ok = warp_wait_bounded(mbar, mk & 1, &g_mxa_err, kErrWaitFull, lane);
-        ++mk;
-        if (!ok) return false;
-      }
-    landed:
+  const int cap = min(16, (int)(land_rows / pbytes));
+  auto issue = [&](int i0, int k) {  // bulk loads of pieces i0 .. i0 + k - 1 into the landing zone
+    fence_proxy_async_smem();  // earlier reads of the landing zone precede the new loads
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(mbar, (uint32_t)k * (pbytes + kRowsPerTile * 4));
       for (int p = 0; p < k; ++p) {
-#pragma unroll
-        for (int q = 0; q < RG; ++q) {
-          const int rr = r0 + q;
-          if (rr >= rows) break;
-          float l;
-          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l) : "r"(land + kLandO + (uint32_t)(p * kRowsPerTile + rr) * 4) : "memory");
-          if (l == -INFINITY) continue;  // an empty piece carries no weight
-          float o[VEC];
-          const uint32_t src = land + (uint32_t)p * pbytes + (uint32_t)(rr * D + col) * 4;
-          if constexpr (VEC == 4) {
-            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(o[0]), "=f"(o[1]), "=f"(o[2]), "=f"(o[3]) : "r"(src) : "memory");
-          } else {
-            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(o[0]), "=f"(o[1]) : "r"(src) : "memory");
-          }
-          const float mn = fmaxf(m[q], l);
-          const float keep = m[q] == -INFINITY ? 0.f : expf(m[q] - mn);
-          const float w = expf(l - mn);
-          ssum[q] = ssum[q] * keep + w;
-#pragma unroll
-          for (int v = 0; v < VEC; ++v) acc[q][v] = acc[q][v] * keep + w * o[v];
-          m[q] = mn;
-        }
+        const size_t sl = slot_of(i0 + p);
+        bulk_load(land + (uint32_t)p * pbytes, a.o_part + sl * kRowsPerTile * D, pbytes, mbar);
+        bulk_load(land + land_rows + (uint32_t)p * kRowsPerTile * 4, a.lse_part + sl * kRowsPerTile,
+                  kRowsPerTile * 4, mbar);
       }
     }
-#pragma unroll
-    for (int q = 0; q < RG; ++q) {
-      const int rr = r0 + q;
-      if (rr < rows) {
-        const float inv = ssum[q] > 0.f ? 1.f / ssum[q] : 0.f;
-        float out_v[VEC];
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) out_v[v] = acc[q][v] * inv;
-        const float lse = m[q] == -INFINITY ? -INFINITY : m[q] + logf(ssum[q]);
-        const int mrow = sg.rt * kRowsPerTile + rr, t = mrow / a.G, g = mrow % a.G, hq = sg.h * a.G + g;
-        stage_out_vec<D, kBf16>(ostage, rr, col, out_v);
-        if (lane == 0 && a.lse != nullptr) a.lse[((size_t)sg.b * a.Hq + hq) * a.q_len + t] = lse;
-      }
+    __syncwarp();
+  };
+  issue(0, min(cap, n));  // the first landing overlaps the row statistics
+
+  // ---- pass 1: per-row maximum and sum of exponentials (base 2) ----
+  const int lpr = rows > 8 ? 2 : rows > 4 ? 4 : rows > 2 ? 8 : rows > 1 ? 16 : 32;  // lanes per row
+  const int r1 = lane / lpr, j1 = lane % lpr;
+  float mx = -INFINITY, sm = 0.f;
+  if (r1 < rows) {
+#pragma unroll 4
+    for (int p = j1; p < n; p += lpr) {
+      // written by other CTAs during this launch: read at L2, past L1
+      const float l = __ldcg(a.lse_part + slot_of(p) * kRowsPerTile + r1) * kLog2e;
+      if (l == -INFINITY) continue;  // an empty piece carries no weight
+      const float mn = fmaxf(mx, l);
+      sm = sm * ex2(mx - mn) + ex2(l - mn);
+      mx = mn;
     }
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    if (o >= lpr) continue;
+    const float mo = __shfl_xor_sync(0xffffffffu, mx, o);
+    const float so = __shfl_xor_sync(0xffffffffu, sm, o);
+    const float mn = fmaxf(mx, mo);
+    sm = (mx == -INFINITY ? 0.f : sm * ex2(mx - mn)) + (mo == -INFINITY ? 0.f : so * ex2(mo - mn));
+    mx = mn;
+  }
+  const float lse2 = sm > 0.f ? mx + log2f(sm) : -INFINITY;  // this row's LSE, base 2
+  if (r1 < rows && j1 == 0 && a.lse != nullptr) {
+    const int mrow = sg.rt * kRowsPerTile + r1, t = mrow / a.G, g = mrow % a.G;
+    a.lse[((size_t)sg.b * a.Hq + (size_t)sg.h * a.G + g) * a.q_len + t] = lse2 * kLn2;
+  }
+  float row_lse[kRowsPerTile];
+#pragma unroll
+  for (int rr = 0; rr < kRowsPerTile; ++rr) row_lse[rr] = __shfl_sync(0xffffffffu, lse2, (rr * lpr) & 31);
+
+  // ---- pass 2: O = sum_i w_i O_i with w_i = exp(lse_i - LSE) ----
+  // All 16 row slots are computed without branches so the loads overlap;
+  // slots past `rows` read a valid row and their sums are never stored.
+  const int col = lane * VEC;
+  const uint32_t sbase = smem_addr(smem);
+  const float *land_o = reinterpret_cast<const float *>(smem + (land - sbase));
+  const float *land_l = reinterpret_cast<const float *>(smem + (land + land_rows - sbase));
+  float acc[kRowsPerTile][VEC];
+#pragma unroll
+  for (int rr = 0; rr < kRowsPerTile; ++rr)
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[rr][v] = 0.f;
+  for (int i0 = 0; i0 < n; i0 += cap) {
+    const int k = min(cap, n - i0);
+    {
+      const bool ok = warp_wait_bounded(mbar, mk & 1, &g_mxa_err, kErrWaitFull, lane);
+      ++mk;
+      if (!ok) return false;
+    }
+    for (int p = 0; p < k; ++p) {
+      const float *lp = land_l + p * kRowsPerTile;
+      const float *op = land_o + p * rows * D + col;
+#pragma unroll
+      for (int rr = 0; rr < kRowsPerTile; ++rr) {
+        const int rc = rr < rows ? rr : rows - 1;
+        const float l = lp[rr] * kLog2e;
+        const float w = l == -INFINITY ? 0.f : ex2(l - row_lse[rr]);
+        if constexpr (VEC == 4) {
+          const float4 v = *reinterpret_cast<const float4 *>(op + rc * D);
+          acc[rr][0] += w * v.x; acc[rr][1] += w * v.y; acc[rr][2] += w * v.z; acc[rr][3] += w * v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2 *>(op + rc * D);
+          acc[rr][0] += w * v.x; acc[rr][1] += w * v.y;
+        }
+      }
+    }
+    if (i0 + cap < n) issue(i0 + cap, min(cap, n - i0 - cap));
+  }
+  __syncwarp();  // every lane is done with the landing zone, which may be the staging buffer
+#pragma unroll
+  for (int rr = 0; rr < kRowsPerTile; ++rr)
+    if (rr < rows) stage_out_vec<D, kBf16>(smem, ostage, rr, col, acc[rr]);
   fence_proxy_async_smem();  // staged rows are read by the bulk stores
   __syncwarp();
   if (lane == 0) {
@@ -909,6 +947,10 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
     const int rows = min(kRowsPerTile, a.M - sg.rt * kRowsPerTile);
     const int unit = (sg.b * a.Hkv + sg.h) * a.RT + sg.rt;
     const int slot = sg.kind - 1;  // partial slot (kind 1 -> head slot 0, kind 2 -> tail slot 1)
+    // a piece of a split unit reads the unit's counter now; the read returns
+    // while this job is processed (it may be stale: the count corrects it)
+    unsigned long long cnt_guess = 0;
+    if (sg.kind != 0 && lane == 0) cnt_guess = __ldcg(a.counters + unit);
 
     // statistics of row `lane`: the four warps' (m, l) merged
     float wgt[kMathWarps];
@@ -936,36 +978,43 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
       for (int w = 0; w < kMathWarps; ++w) wgt[w] *= inv;
       my_lse = Lx > 0.f ? (Mx + log2f(Lx)) * kLn2 : NEG_INF;
     }
-    for (int rr = 0; rr < rows; ++rr) {
-      float acc[VEC];
+    // O of each row: the four warps' unnormalised partials, weighted.  A
+    // warp whose weight is 0 left zeros (or finite values) in its slice, so
+    // every load is made.  All 16 row slots are loaded before anything is
+    // staged and without branches, so the loads overlap; slots past `rows`
+    // read a valid row and are never stored.
+    const float *hbase = reinterpret_cast<const float *>(smem + (sbase - smem_addr(smem)));
+    float acc[kRowsPerTile][VEC];
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+    for (int rr = 0; rr < kRowsPerTile; ++rr) {
+      const int rc = rr < rows ? rr : rows - 1;
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[rr][v] = 0.f;
 #pragma unroll
       for (int w = 0; w < kMathWarps; ++w) {
         const float wg = __shfl_sync(0xffffffffu, wgt[w], rr);
-        if (wg != 0.f) {
-          const uint32_t addr = handoff_addr<D>(sbase, w, rr, col);
-          if constexpr (VEC == 4) {
-            float4 v;
-            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                         : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
-            acc[0] += wg * v.x; acc[1] += wg * v.y; acc[2] += wg * v.z; acc[3] += wg * v.w;
-          } else {
-            float2 v;
-            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
-            acc[0] += wg * v.x; acc[1] += wg * v.y;
-          }
+        const float *src = hbase + (handoff_addr<D>(sbase, w, rc, col) - sbase) / 4;
+        if constexpr (VEC == 4) {
+          const float4 v = *reinterpret_cast<const float4 *>(src);
+          acc[rr][0] += wg * v.x; acc[rr][1] += wg * v.y; acc[rr][2] += wg * v.z; acc[rr][3] += wg * v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2 *>(src);
+          acc[rr][0] += wg * v.x; acc[rr][1] += wg * v.y;
         }
       }
-      if (sg.kind == 0) {
-        stage_out_vec<D, kBf16>(ostage, rr, col, acc);
-      } else {  // fp32 partial rows, pitch D * 4 bytes
-        const uint32_t addr = ostage + (uint32_t)(rr * D + col) * 4;
-        if constexpr (VEC == 4) {
-          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(acc[0]), "f"(acc[1]),
-                       "f"(acc[2]), "f"(acc[3]) : "memory");
-        } else {
-          asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(acc[0]), "f"(acc[1]) : "memory");
+    }
+#pragma unroll
+    for (int rr = 0; rr < kRowsPerTile; ++rr) {
+      if (rr < rows) {
+        if (sg.kind == 0) {
+          stage_out_vec<D, kBf16>(smem, ostage, rr, col, acc[rr]);
+        } else {  // fp32 partial rows, pitch D * 4 bytes
+          float *dst = reinterpret_cast<float *>(smem + (ostage - smem_addr(smem))) + rr * D + col;
+          if constexpr (VEC == 4) {
+            *reinterpret_cast<float4 *>(dst) = make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
+          } else {
+            *reinterpret_cast<float2 *>(dst) = make_float2(acc[rr][0], acc[rr][1]);
+          }
         }
       }
     }
@@ -1007,11 +1056,11 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
       __threadfence();
       __syncwarp();
       bool ok = true;
-      if (arrive_and_check_last(a, unit, sg.n_pieces, lane)) {
+      if (arrive_and_check_last(a, unit, sg.n_pieces, lane, cnt_guess)) {
         __threadfence();
-        ok = hold ? merge_pieces<D, kBf16>(a, sg, rows, unit, lane, ostage, sbase, stage_land_rows<D>(),
+        ok = hold ? merge_pieces<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, sbase, stage_land_rows<D>(),
                                            merge_bar, mk)
-                  : merge_pieces<D, kBf16>(a, sg, rows, unit, lane, ostage, oland, (uint32_t)kLandRows,
+                  : merge_pieces<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, oland, (uint32_t)kLandRows,
                                            merge_bar, mk);
       }
       if (hold) {
@@ -1212,6 +1261,7 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
   a.chunk_blocks = plan.schedule == MXA_SCHED_UNIFORM ? (max_blocks + plan.num_splits - 1) / plan.num_splits : 1;
   if (a.chunk_blocks < 1) a.chunk_blocks = 1;
   a.units = plan.units;
+  a.unit_cost = plan.schedule == MXA_SCHED_BALANCED ? plan.unit_cost : 0;
   a.epoch = next_epoch();
   if (plan.workspace_bytes > 0) {
     uint8_t *ws = static_cast<uint8_t *>(L.workspace);

@@ -38,6 +38,7 @@ struct DecodeArgs {
   int splits;                  // UNIFORM: splits per unit
   int chunk_blocks;            // UNIFORM: blocks per split
   int units;
+  int unit_cost;               // BALANCED: fixed cost of a unit, in KV blocks
   unsigned int epoch;          // tags this launch's arrival counts
 };
 

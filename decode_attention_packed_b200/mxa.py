@@ -45,7 +45,7 @@ class mxa_plan_t(ctypes.Structure):
                 ("units", ctypes.c_int), ("rows_per_tile", ctypes.c_int),
                 ("block_tokens", ctypes.c_int), ("ctas_per_sm", ctypes.c_int),
                 ("sm_count", ctypes.c_int), ("needs_combine", ctypes.c_int),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("unit_cost", ctypes.c_int), ("workspace_bytes", ctypes.c_size_t)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}

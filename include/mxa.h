@@ -65,13 +65,16 @@ typedef enum { MXA_F16 = 0, MXA_BF16 = 1 } mxa_dtype_t;
  *           multiples of one chunk, chunk = ceil(max_seqlen_k / num_splits)
  *           tokens rounded up to the pipeline block; grid = units * num_splits.
  *           num_splits = 1 means one CTA per unit and no combine pass.
- * BALANCED: the KV blocks of all units, laid end to end (unit-major), are
+ * BALANCED: the work of all units, laid end to end (unit-major), is
  *           divided into `grid` equal contiguous ranges, one per CTA; a unit
- *           that straddles ranges is merged by the combine pass.  Every CTA
- *           streams the same number of KV bytes however ragged the lengths
- *           are (a length-aware split in the spirit of the cost-balanced
- *           core assignment of "MixedQuantSparseFlashMlaMetadata 算子解析",
- *           section 源码级原理). */
+ *           that straddles ranges is merged by the combine pass.  A unit's
+ *           work is its KV blocks plus a fixed cost of `unit_cost` blocks
+ *           (its query load, the merge of its warps' results and its output
+ *           stores), so every CTA gets the same work however ragged the
+ *           lengths are (a length-aware split in the spirit of the
+ *           cost-balanced core assignment of "MixedQuantSparseFlashMlaMetadata
+ *           算子解析", section 源码级原理, which also charges each task a fixed
+ *           cost besides its KV length). */
 typedef enum { MXA_SCHED_UNIFORM = 0, MXA_SCHED_BALANCED = 1 } mxa_schedule_t;
 
 /* Problem shape.
@@ -107,6 +110,8 @@ typedef struct {
   int ctas_per_sm;       /* resident CTAs per SM the plan assumed */
   int sm_count;          /* SMs the plan assumed */
   int needs_combine;     /* 1 if units may be split across CTAs and merged (needs the workspace) */
+  int unit_cost;         /* BALANCED: fixed cost of a unit, in KV blocks, added to its blocks
+                            when the work is divided (0..64); UNIFORM: unused */
   size_t workspace_bytes;/* device scratch the run needs (0 if none) */
 } mxa_plan_t;
 
@@ -145,7 +150,7 @@ MXA_API int mxa_num_splits_heuristic(int tiles, int sm_count, int slots, int num
  *                    efficiency optimum when every CTA carries the same
  *                    work), capped at units * ceil(blocks per unit / 4) so
  *                    no unit is cut into pieces under 4 blocks on average;
- *                    for B above 16384 rows, UNIFORM with s from
+ *                    for B above 12288 rows, UNIFORM with s from
  *                    mxa_num_splits_heuristic.
  *   sm_count > 0   : plan for that many SMs (pure host computation);
  *   sm_count <= 0  : query the current CUDA device (MXA_ERR_CUDA without one).
@@ -164,7 +169,7 @@ MXA_API mxa_status_t mxa_plan(const mxa_decode_params_t *params, int num_splits,
  * the split and for tests: the same as mxa_plan's automatic plan with its
  * grid replaced.  Pure host computation apart from sm_count <= 0, which
  * queries the current device.  Errors as mxa_plan; MXA_ERR_UNSUPPORTED if
- * B exceeds the 16384 rows the balanced prologue scans. */
+ * B exceeds the 12288 rows the balanced prologue scans. */
 MXA_API mxa_status_t mxa_plan_balanced(const mxa_decode_params_t *params, int grid, int sm_count,
                                        mxa_plan_t *plan);
 
@@ -192,7 +197,7 @@ MXA_API mxa_status_t mxa_decode_fwd(const void *q, const void *k_cache, const vo
 /* As mxa_decode_fwd, but run a plan the caller resolved (or built) before:
  * the second phase of the two-phase call.  The plan is validated against
  * `params` (schedule, grid >= 1, units, block_tokens); a BALANCED plan may
- * use any grid >= 1. */
+ * use any grid >= 1 and any unit_cost in 0..64. */
 MXA_API mxa_status_t mxa_decode_fwd_with_plan(const void *q, const void *k_cache, const void *v_cache,
                                       const int32_t *block_table, const int32_t *cache_seqlens,
                                       const mxa_decode_params_t *params, float scale, int causal,

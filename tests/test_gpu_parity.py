@@ -108,6 +108,31 @@ def test_ragged_balanced_grids(grid):
     check(inp, out, lse, ref)
 
 
+@pytest.mark.parametrize("unit_cost", [0, 1, 5, 64])
+@pytest.mark.parametrize("grid", [3, 296, 1500])
+def test_balanced_unit_costs(grid, unit_cost):
+    # the fixed cost per unit moves every range boundary; every block must
+    # still be read exactly once and every split unit merged
+    inp, ref, dev = full(4)
+    q, k, v, bt, sl = dev
+    plan = mxa.mxa_plan_balanced(mxa.params_for(q, k, bt, inp.max_seqlen_k), grid)
+    plan.unit_cost = unit_cost
+    out, lse, _ = run_gpu(inp, plan=plan, dev=dev)
+    check(inp, out, lse, ref)
+
+
+@pytest.mark.parametrize("unit_cost", [0, 3, 64])
+def test_balanced_unit_costs_edge_lengths(unit_cost):
+    # rows of every length class, including L = 0 rows that hold no unit
+    inp = make_inputs(wl())
+    dev = to_dev(inp)
+    q, k, v, bt, sl = dev
+    plan = mxa.mxa_plan_balanced(mxa.params_for(q, k, bt, inp.max_seqlen_k), 37)
+    plan.unit_cost = unit_cost
+    out, lse, _ = run_gpu(inp, plan=plan, dev=dev)
+    check(inp, out, lse)
+
+
 # --------------------------------------------------------------------------
 # shapes and edges at sizes the oracle finishes in seconds
 # --------------------------------------------------------------------------

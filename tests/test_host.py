@@ -98,6 +98,10 @@ def test_plan_long_context_split():
     assert plan.units == 16 and plan.grid == 296 and plan.num_splits == 19
     assert plan.ctas_per_sm == 2 and plan.block_tokens == 64
     assert plan.needs_combine == 1 and plan.workspace_bytes > 0
+    # each unit is charged a fixed cost of two blocks besides its KV blocks
+    assert plan.unit_cost == 2
+    assert mxa.mxa_plan_balanced(params(), 100, sm_count=148).unit_cost == 2
+    assert mxa.mxa_plan(params(), 3, sm_count=148).unit_cost == 0
 
 
 def test_plan_does_not_split_tiny_problems():
@@ -170,6 +174,11 @@ def test_run_refuses_bad_arguments_before_launch():
     bad = mxa.mxa_plan(p, 2, sm_count=148)
     bad.grid += 1
     assert _run_with_plan(p, bad, ws=1, ws_bytes=1 << 30) == MXA_ERR_INVALID_ARG
+    # a balanced plan's fixed unit cost must lie in 0..64
+    for cost in (-1, 65):
+        bad = mxa.mxa_plan(p, 0, sm_count=148)
+        bad.unit_cost = cost
+        assert _run_with_plan(p, bad, ws=1, ws_bytes=1 << 30) == MXA_ERR_INVALID_ARG
     # nothing to do for B = 0
     p0 = params(B=0)
     assert _run_with_plan(p0, mxa.mxa_plan(p0, 1, sm_count=148)) == MXA_OK

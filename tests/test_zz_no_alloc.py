@@ -73,10 +73,10 @@ def test_noalloc_matches_workspace_entry_point(i):
 
 
 def test_noalloc_refuses_plans_beyond_its_array():
-    # 2048 units with a balanced grid of 2048 CTAs need ~34 MB of split scratch
+    # 2048 units cut into 8 uniform splits: 16384 CTAs, ~268 MB of split scratch
     params = mxa.mxa_decode_params_t(256, 1, 64, 8, 128, 65536, 16, 256, 4096, mxa.MXA_BF16)
-    plan = mxa.mxa_plan(params, 0)
+    plan = mxa.mxa_plan(params, 8)
     assert plan.workspace_bytes > 16 << 20
     rc = mxa._lib.mxa_decode_fwd_noalloc(None, None, None, None, None, ctypes.byref(params), 0.088, 0,
-                                         0, None, None, _stream())
+                                         8, None, None, _stream())
     assert rc == mxa.MXA_ERR_WORKSPACE
