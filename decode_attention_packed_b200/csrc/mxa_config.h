@@ -53,8 +53,11 @@ struct JobSlot {
   float ml[kMathWarps][kRowsPerTile][2];
 };
 
-constexpr size_t kBarrierBytes = 128;   // full[S], empty[S], qfull, qempty, job_full[J], job_empty[J], merge
-constexpr int kNumBarriers = 2 * kStages + 2 + 2 * kJobs + 1;
+// full[S], empty[S], qfull, qempty, job_full[J], job_empty[J], merge, init;
+// then the two split units whose counters the CTA tags (2 ints)
+constexpr size_t kBarrierBytes = 128;
+constexpr int kNumBarriers = 2 * kStages + 2 + 2 * kJobs + 2;
+constexpr size_t kInitUnitsOff = (size_t)kNumBarriers * 8;
 
 // Offsets inside the dynamic shared memory (base aligned to 1024 bytes).
 constexpr size_t smem_ring_off() { return 0; }
@@ -90,7 +93,7 @@ inline size_t workspace_bytes(long units, long grid, int D) {
   return ws_count_bytes(units) + ws_lse_bytes(grid) + ws_o_bytes(grid, D);
 }
 
-static_assert(kNumBarriers * 8 <= (int)kBarrierBytes, "barrier area");
+static_assert(kInitUnitsOff + 2 * sizeof(int) <= kBarrierBytes, "barrier area");
 static_assert(sizeof(SegmentDesc) % 16 == 0 && sizeof(JobSlot) % 16 == 0, "alignment");
 static_assert(2 * (smem_total(128) + kSmemReservedPerCta) <= (size_t)kSmemPerSm,
               "D = 128 layout must leave room for two CTAs per SM");

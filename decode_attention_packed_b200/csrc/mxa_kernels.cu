@@ -57,6 +57,7 @@ constexpr int B_QEMPTY = 2 * kStages + 1;
 constexpr int B_JOBFULL(int j) { return 2 * kStages + 2 + j; }
 constexpr int B_JOBEMPTY(int j) { return 2 * kStages + 2 + kJobs + j; }
 constexpr int B_MERGE = 2 * kStages + 2 + 2 * kJobs;  // pieces of a split unit landed by bulk loads
+constexpr int B_INIT = B_MERGE + 1;                     // the producer has published the CTA's split units
 
 // ---------------------------------------------------------------------------
 // Producer warp
@@ -286,6 +287,22 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
   bool has_tail;
   Cursor cur = cursor_start<D>(a, smem, lane, tail, has_tail);
   auto more = [&]() { return has_tail || (cur.x < cur.end && cur.nb > 0); };
+  // Publish the units of this CTA that are split across CTAs (at most the
+  // first unit of its range and the tail unit): the epilogue warp tags their
+  // arrival counters with this launch's epoch before any piece is counted.
+  if (lane == 0) {
+    const int HR = a.Hkv * a.RT;
+    int u_first = -1;
+    if (cur.x < cur.end && cur.nb > 0) {
+      const bool split = a.schedule == MXA_SCHED_BALANCED ? (cur.blk > 0 || cur.x - cur.blk + cur.nb > cur.end)
+                                                          : cur.nb > a.chunk_blocks;
+      if (split) u_first = cur.b * HR + cur.hr;
+    }
+    int *init_units = reinterpret_cast<int *>(smem + smem_bar_off(D) + kInitUnitsOff);
+    init_units[0] = u_first;
+    init_units[1] = has_tail ? tail.b * HR + tail.hr : -1;
+    mbar_arrive(bar_addr(smem, D, B_INIT));
+  }
   auto take = [&]() {
     if (has_tail) {
       has_tail = false;
@@ -747,27 +764,6 @@ __device__ void write_empty_unit(const DecodeArgs &a, int unit, int lane) {
   __syncwarp();
 }
 
-// Count this piece of a split unit; true (in every lane) for the piece that
-// completes it.  The counter carries the call's epoch in its high half, so a
-// count left by an earlier (failed) call is not mistaken for this call's.
-// `guess` is lane 0's earlier read of the counter: when no other piece has
-// arrived since, the first compare-and-swap succeeds.  The retry loop runs
-// on all lanes; only lane 0 touches memory.
-__device__ __forceinline__ bool arrive_and_check_last(const DecodeArgs &a, int unit, int n, int lane,
-                                                      unsigned long long guess) {
-  unsigned long long *cnt = a.counters + unit;
-  const unsigned long long ep = a.epoch;
-  unsigned long long cur = __shfl_sync(0xffffffffu, guess, 0);
-  for (;;) {
-    const unsigned long long want = (cur >> 32) == ep ? cur + 1ull : ((ep << 32) | 1ull);
-    unsigned long long prev = 0;
-    if (lane == 0) prev = atomicCAS(cnt, cur, want);
-    prev = __shfl_sync(0xffffffffu, prev, 0);
-    if (prev == cur) return (int)(want & 0xffffffffull) == n;
-    cur = prev;
-  }
-}
-
 // Room for partial rows in a landing zone that is a whole ring stage; its
 // LSEs follow.
 template <int D>
@@ -775,57 +771,79 @@ constexpr uint32_t stage_land_rows() { return (uint32_t)stage_bytes(D) - 16 * kR
 
 // Merge the n pieces of a split unit with the log-sum-exp identity,
 // LSE = ln sum_i exp(lse_i) and O = sum_i exp(lse_i - LSE) O_i, in two
-// passes.  First the row statistics: the pieces' LSEs are read straight
-// from global memory, spread over a power-of-two group of lanes per row,
-// and reduced with a running maximum.  Then the weighted sum: the pieces'
-// partial rows and LSEs are brought into a landing zone (`land`, with
-// `land_rows` bytes for rows and the LSEs after them) with bulk loads, up
-// to 16 pieces at a time, and every lane accumulates its D / 32 columns of
-// every row.  With the weights known up front the products are independent
-// of one another, so the loads of many rows and pieces overlap.  The
+// passes.  The pieces' partial rows and LSEs are brought into a landing zone
+// (`land`, with `land_rows` bytes for rows and the LSEs after them) with
+// bulk loads, up to 16 pieces' rows at a time; the LSEs of all pieces come
+// with the first landing when there are at most 16 pieces (else each batch
+// brings its own and the row statistics read them from global memory).
+// First the row statistics, spread over a power-of-two group of lanes per
+// row and reduced with a running maximum; then every lane accumulates its
+// D / 32 columns of every row with the weights known up front, so the
+// products are independent of one another and the loads overlap.  The
 // pieces are the tail slot of the first CTA and the head slots of the
-// following ones.  Returns false if a bounded wait ran out.
+// following ones.  The caller has acquired their writes (the arrival
+// count).  `own` >= 0 names a piece the caller has already placed in the
+// landing zone (rows and LSEs at its index; then all n pieces fit one
+// landing).  Returns false if a bounded wait ran out.
 template <int D, bool kBf16>
 __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int rows, int unit, int lane,
                              uint8_t *smem, uint32_t ostage, uint32_t land, uint32_t land_rows,
-                             uint32_t mbar, uint32_t &mk) {
+                             uint32_t mbar, uint32_t &mk, int own) {
   constexpr int VEC = D / 32;
   constexpr float kLog2e = 1.4426950408889634f;
   const int n = sg.n_pieces, cf = sg.c_first;
   auto slot_of = [&](int i) -> size_t { return i == 0 ? (size_t)cf * 2 + 1 : (size_t)(cf + i) * 2; };
-
   const uint32_t pbytes = (uint32_t)rows * D * 4;
-  const int cap = min(16, (int)(land_rows / pbytes));
-  auto issue = [&](int i0, int k) {  // bulk loads of pieces i0 .. i0 + k - 1 into the landing zone
+  const int cap = min(kRowsPerTile, (int)(land_rows / pbytes));
+  const bool all_lse = n <= kRowsPerTile;  // every piece's LSEs come with the first landing
+  auto issue = [&](int i0, int k) {  // bulk loads of pieces i0 .. i0 + k - 1
     fence_proxy_async_smem();  // earlier reads of the landing zone precede the new loads
     __syncwarp();
     if (lane == 0) {
-      mbar_arrive_expect_tx(mbar, (uint32_t)k * (pbytes + kRowsPerTile * 4));
-      for (int p = 0; p < k; ++p) {
-        const size_t sl = slot_of(i0 + p);
-        bulk_load(land + (uint32_t)p * pbytes, a.o_part + sl * kRowsPerTile * D, pbytes, mbar);
-        bulk_load(land + land_rows + (uint32_t)p * kRowsPerTile * 4, a.lse_part + sl * kRowsPerTile,
-                  kRowsPerTile * 4, mbar);
-      }
+      const int l0 = all_lse ? 0 : i0, nl = all_lse ? (i0 == 0 ? n : 0) : k;
+      const int ko = (own >= i0 && own < i0 + k) ? 1 : 0, lo = (own >= l0 && own < l0 + nl) ? 1 : 0;
+      mbar_arrive_expect_tx(mbar, (uint32_t)(k - ko) * pbytes + (uint32_t)(nl - lo) * kRowsPerTile * 4);
+      for (int p = 0; p < k; ++p)
+        if (i0 + p != own)
+          bulk_load(land + (uint32_t)p * pbytes, a.o_part + slot_of(i0 + p) * kRowsPerTile * D, pbytes, mbar);
+      for (int p = 0; p < nl; ++p)
+        if (l0 + p != own)
+          bulk_load(land + land_rows + (uint32_t)p * kRowsPerTile * 4, a.lse_part + slot_of(l0 + p) * kRowsPerTile,
+                    kRowsPerTile * 4, mbar);
     }
     __syncwarp();
   };
-  issue(0, min(cap, n));  // the first landing overlaps the row statistics
+  auto landed = [&]() {
+    const bool ok = warp_wait_bounded(mbar, mk & 1, &g_mxa_err, kErrWaitFull, lane);
+    ++mk;
+    return ok;
+  };
+  if (lane == 0) fence_proxy_async_global();  // the acquired writes precede these async-proxy reads
+  __syncwarp();
+  issue(0, min(cap, n));
+
+  const uint32_t sbase = smem_addr(smem);
+  const float *land_o = reinterpret_cast<const float *>(smem + (land - sbase));
+  const float *land_l = reinterpret_cast<const float *>(smem + (land + land_rows - sbase));
 
   // ---- pass 1: per-row maximum and sum of exponentials (base 2) ----
   const int lpr = rows > 8 ? 2 : rows > 4 ? 4 : rows > 2 ? 8 : rows > 1 ? 16 : 32;  // lanes per row
   const int r1 = lane / lpr, j1 = lane % lpr;
   float mx = -INFINITY, sm = 0.f;
-  if (r1 < rows) {
+  auto take_lse = [&](float l) {
+    if (l == -INFINITY) return;  // an empty piece carries no weight
+    const float mn = fmaxf(mx, l);
+    sm = sm * ex2(mx - mn) + ex2(l - mn);
+    mx = mn;
+  };
+  if (!all_lse && r1 < rows) {
 #pragma unroll 4
-    for (int p = j1; p < n; p += lpr) {
-      // written by other CTAs during this launch: read at L2, past L1
-      const float l = __ldcg(a.lse_part + slot_of(p) * kRowsPerTile + r1) * kLog2e;
-      if (l == -INFINITY) continue;  // an empty piece carries no weight
-      const float mn = fmaxf(mx, l);
-      sm = sm * ex2(mx - mn) + ex2(l - mn);
-      mx = mn;
-    }
+    for (int p = j1; p < n; p += lpr)  // read at L2, past L1: written during this launch
+      take_lse(__ldcg(a.lse_part + slot_of(p) * kRowsPerTile + r1) * kLog2e);
+  }
+  if (!landed()) return false;
+  if (all_lse && r1 < rows) {
+    for (int p = j1; p < n; p += lpr) take_lse(land_l[p * kRowsPerTile + r1] * kLog2e);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -849,9 +867,6 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
   // All 16 row slots are computed without branches so the loads overlap;
   // slots past `rows` read a valid row and their sums are never stored.
   const int col = lane * VEC;
-  const uint32_t sbase = smem_addr(smem);
-  const float *land_o = reinterpret_cast<const float *>(smem + (land - sbase));
-  const float *land_l = reinterpret_cast<const float *>(smem + (land + land_rows - sbase));
   float acc[kRowsPerTile][VEC];
 #pragma unroll
   for (int rr = 0; rr < kRowsPerTile; ++rr)
@@ -859,13 +874,9 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
     for (int v = 0; v < VEC; ++v) acc[rr][v] = 0.f;
   for (int i0 = 0; i0 < n; i0 += cap) {
     const int k = min(cap, n - i0);
-    {
-      const bool ok = warp_wait_bounded(mbar, mk & 1, &g_mxa_err, kErrWaitFull, lane);
-      ++mk;
-      if (!ok) return false;
-    }
+    if (i0 > 0 && !landed()) return false;
     for (int p = 0; p < k; ++p) {
-      const float *lp = land_l + p * kRowsPerTile;
+      const float *lp = land_l + (all_lse ? i0 + p : p) * kRowsPerTile;
       const float *op = land_o + p * rows * D + col;
 #pragma unroll
       for (int rr = 0; rr < kRowsPerTile; ++rr) {
@@ -921,6 +932,24 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
     if (clamp_len(a.seqlens[u / HR], a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, lane);
   }
 
+  // Tag the arrival counters of this CTA's split units with this launch's
+  // epoch (count 0), unless a piece in another CTA already did: every piece
+  // of a unit does this before it can arrive, so arrivals are plain atomic
+  // adds and a stale count (an earlier call's, or garbage) is never added
+  // to.  A failed compare-and-swap means another CTA has tagged it.
+  if (!warp_wait_bounded(bar_addr(smem, D, B_INIT), 0, &g_mxa_err, kErrWaitQ, lane)) return;
+  if (lane == 0) {
+    const int *init_units = reinterpret_cast<const int *>(smem + smem_bar_off(D) + kInitUnitsOff);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int u = init_units[i];
+      if (u >= 0) {
+        unsigned long long *cnt = a.counters + u;
+        const unsigned long long cur = ld_relaxed_gpu_u64(cnt);
+        if ((cur >> 32) != (unsigned long long)a.epoch) atomicCAS(cnt, cur, (unsigned long long)a.epoch << 32);
+      }
+    }
+  }
   const int col = lane * VEC;
   const uint32_t ostage = smem_addr(smem + smem_out_off(D));
   const uint32_t oland = ostage;  // free again once this job's own rows have been stored
@@ -947,10 +976,12 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
     const int rows = min(kRowsPerTile, a.M - sg.rt * kRowsPerTile);
     const int unit = (sg.b * a.Hkv + sg.h) * a.RT + sg.rt;
     const int slot = sg.kind - 1;  // partial slot (kind 1 -> head slot 0, kind 2 -> tail slot 1)
-    // a piece of a split unit reads the unit's counter now; the read returns
-    // while this job is processed (it may be stale: the count corrects it)
-    unsigned long long cnt_guess = 0;
-    if (sg.kind != 0 && lane == 0) cnt_guess = __ldcg(a.counters + unit);
+    // A piece of a split unit reads the unit's count now (acquire); the read
+    // completes while this job is merged.  If every other piece has already
+    // arrived, this piece merges the unit at once: it neither stores its
+    // own partial nor counts itself.
+    unsigned long long seen = 0;
+    if (sg.kind != 0 && lane == 0) seen = ld_acquire_gpu_u64(a.counters + unit);
 
     // statistics of row `lane`: the four warps' (m, l) merged
     float wgt[kMathWarps];
@@ -1003,13 +1034,26 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
         }
       }
     }
+    // A split unit's landing zone: the staging buffer when all its pieces'
+    // rows fit there, else the ring stage this job came in (kept until the
+    // piece has been counted, and merged if it was the last).
+    const bool hold = sg.kind != 0 && (uint32_t)sg.n_pieces * rows * D * 4 > (uint32_t)kLandRows;
+    const uint32_t land = hold ? sbase : oland;
+    const uint32_t land_rows = hold ? stage_land_rows<D>() : (uint32_t)kLandRows;
+    const int own = (int)blockIdx.x - sg.c_first;  // this piece's index in the unit
+    seen = __shfl_sync(0xffffffffu, seen, 0);
+    const bool merge_now = sg.kind != 0 && (seen >> 32) == (unsigned long long)a.epoch &&
+                           (int)(seen & 0xffffffffull) == sg.n_pieces - 1 &&
+                           sg.n_pieces <= min(kRowsPerTile, (int)(land_rows / ((uint32_t)rows * D * 4)));
+    __syncwarp();  // every lane has read the stage before it may become the landing zone
+    const uint32_t dst_rows = merge_now ? land + (uint32_t)own * rows * D * 4 : ostage;
 #pragma unroll
     for (int rr = 0; rr < kRowsPerTile; ++rr) {
       if (rr < rows) {
         if (sg.kind == 0) {
           stage_out_vec<D, kBf16>(smem, ostage, rr, col, acc[rr]);
         } else {  // fp32 partial rows, pitch D * 4 bytes
-          float *dst = reinterpret_cast<float *>(smem + (ostage - smem_addr(smem))) + rr * D + col;
+          float *dst = reinterpret_cast<float *>(smem + (dst_rows - smem_addr(smem))) + rr * D + col;
           if constexpr (VEC == 4) {
             *reinterpret_cast<float4 *>(dst) = make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
           } else {
@@ -1023,8 +1067,10 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
       if (sg.kind == 0) {
         const int m = sg.rt * kRowsPerTile + lane, t = m / a.G, g = m % a.G, hq = sg.h * a.G + g;
         if (a.lse != nullptr) a.lse[((size_t)sg.b * a.Hq + hq) * a.q_len + t] = my_lse;
-      } else {
-        a.lse_part[((size_t)blockIdx.x * 2 + slot) * kRowsPerTile + lane] = my_lse;
+      } else if (merge_now) {  // at this piece's index among the landed LSEs
+        reinterpret_cast<float *>(smem + (land + land_rows - smem_addr(smem)))[own * kRowsPerTile + lane] = my_lse;
+      } else {  // after the 16 staged rows; stored with them
+        reinterpret_cast<float *>(smem + (ostage - smem_addr(smem)))[kRowsPerTile * D + lane] = my_lse;
       }
     }
     // Give the stage back to the producer and the hand-off slot to the math
@@ -1033,35 +1079,36 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
     // rows out with bulk stores.
     fence_proxy_async_smem();  // staged rows are read by the bulk stores
     __syncwarp();
-    // A merge whose pieces all fit the landing buffer does not need the
-    // stage; otherwise the stage is kept as the landing zone until this
-    // piece has been counted (and merged, if it was the last).
-    const bool hold = sg.kind != 0 && (uint32_t)sg.n_pieces * rows * D * 4 > (uint32_t)kLandRows;
     if (lane == 0) {
       mbar_arrive(bar_addr(smem, D, B_JOBEMPTY(j)));
       if (!hold) mbar_arrive_cnt(bar_addr(smem, D, B_EMPTY(stage)), kMathWarps);
       if (sg.kind == 0) {
         store_out_rows<D>(a, sg.b, sg.h, sg.rt, rows, ostage);
-      } else {
-        bulk_store(a.o_part + ((size_t)blockIdx.x * 2 + slot) * kRowsPerTile * D, ostage, (uint32_t)(rows * D * 4));
+      } else if (!merge_now) {
+        const size_t ps = (size_t)blockIdx.x * 2 + slot;
+        bulk_store(a.o_part + ps * kRowsPerTile * D, ostage, (uint32_t)(rows * D * 4));
+        bulk_store(a.lse_part + ps * kRowsPerTile, ostage + (uint32_t)(kRowsPerTile * D * 4), kRowsPerTile * 4);
       }
       bulk_commit();
     }
     if (sg.kind != 0) {
       // A piece of a split unit: the last piece to arrive merges them all.
-      if (lane == 0) {
-        bulk_wait_all();  // this piece's partial rows are in global memory
-        bulk_wait_read_all();
-      }
-      __threadfence();
-      __syncwarp();
+      // Count it with an acquire-release add: the release publishes this
+      // piece's rows and LSEs (written by the async proxy, completed and
+      // fenced first); the acquire lets the last piece read everyone's.
       bool ok = true;
-      if (arrive_and_check_last(a, unit, sg.n_pieces, lane, cnt_guess)) {
-        __threadfence();
-        ok = hold ? merge_pieces<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, sbase, stage_land_rows<D>(),
-                                           merge_bar, mk)
-                  : merge_pieces<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, oland, (uint32_t)kLandRows,
-                                           merge_bar, mk);
+      if (merge_now) {
+        ok = merge_pieces<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, merge_bar, mk, own);
+      } else {
+        unsigned long long old = 0;
+        if (lane == 0) {
+          bulk_wait_all();  // this piece's partial rows and LSEs are in global memory
+          fence_proxy_async_global();
+          old = atom_add_acq_rel_gpu_u64(a.counters + unit, 1ull);
+        }
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if ((int)(old & 0xffffffffull) + 1 == sg.n_pieces)
+          ok = merge_pieces<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, merge_bar, mk, -1);
       }
       if (hold) {
         fence_proxy_async_smem();  // reads of the landing zone precede the stage's next TMA loads
@@ -1100,6 +1147,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(bar_addr(smem, D, B_JOBEMPTY(j)), 1);
     }
     mbar_init(bar_addr(smem, D, B_MERGE), 1);
+    mbar_init(bar_addr(smem, D, B_INIT), 1);
     fence_mbar_init();
   }
   __syncthreads();
