@@ -40,7 +40,8 @@ struct SegmentDesc {
                          // 2 = tail piece (slot 1), -1 = end of work
   int c_first;           // first CTA holding a piece of the unit
   int n_pieces;          // CTAs holding pieces of the unit
-  int pad[3];
+  int last;              // 1 if no segment follows in this CTA
+  int pad[2];
 };
 
 // What the math warps hand to the epilogue warp at the end of a segment:

@@ -58,6 +58,7 @@ constexpr int B_JOBFULL(int j) { return 2 * kStages + 2 + j; }
 constexpr int B_JOBEMPTY(int j) { return 2 * kStages + 2 + kJobs + j; }
 constexpr int B_MERGE = 2 * kStages + 2 + 2 * kJobs;  // pieces of a split unit landed by bulk loads
 constexpr int B_INIT = B_MERGE + 1;                     // the producer has published the CTA's split units
+constexpr int kRingLseSlots = 32;                       // pieces' LSEs a merge landing in the ring holds
 
 // ---------------------------------------------------------------------------
 // Producer warp
@@ -109,7 +110,8 @@ __device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
     s.c_first = unit * a.splits;
     s.n_pieces = (c.nb + a.chunk_blocks - 1) / a.chunk_blocks;
   }
-  s.pad[0] = s.pad[1] = s.pad[2] = 0;
+  s.last = 0;
+  s.pad[0] = s.pad[1] = 0;
 
   c.x += len;
   c.blk += len;
@@ -342,6 +344,7 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
   bool ok = true;
   if (more()) {
     SegmentDesc seg = take();
+    seg.last = more() ? 0 : 1;
     Window win;
     load_window(seg, win);
     if (!warp_wait_bounded(qempty, 1, &g_mxa_err, kErrWaitQ, lane)) ok = false;  // first use: free
@@ -402,6 +405,7 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
           have_next = more();
           if (have_next) {
             nseg = take();
+            nseg.last = more() ? 0 : 1;
             load_window(nseg, nwin);
           }
         }
@@ -492,7 +496,7 @@ __device__ void math_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lan
   for (;;) {
     if (!warp_wait_bounded(qfull, seg_k & 1, &g_mxa_err, kErrWaitQ, lane)) return;
     const int b = desc[0], h = desc[1], rt = desc[2], blk_beg = desc[3], blk_end = desc[4];
-    const int L = desc[5], kind = desc[6], c_first = desc[7], n_pieces = desc[8];
+    const int L = desc[5], kind = desc[6], c_first = desc[7], n_pieces = desc[8], last = desc[9];
     const int j = seg_k % kJobs, jk = seg_k / kJobs;
     if (kind < 0) {  // end of work: pass the marker on to the epilogue warp
       if (!warp_wait_bounded(bar_addr(smem, D, B_JOBEMPTY(j)), (jk & 1) ^ 1, &g_mxa_err, kErrWaitQ, lane))
@@ -689,7 +693,8 @@ __device__ void math_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lan
       SegmentDesc sd;
       sd.b = b; sd.h = h; sd.rt = rt; sd.blk_beg = blk_beg; sd.blk_end = blk_end; sd.L = L;
       sd.kind = kind; sd.c_first = c_first; sd.n_pieces = n_pieces;
-      sd.pad[0] = sd.pad[1] = sd.pad[2] = 0;
+      sd.last = last;
+      sd.pad[0] = sd.pad[1] = 0;
       jobs[j].seg = sd;
       jobs[j].stage = s_last;
     }
@@ -772,10 +777,11 @@ constexpr uint32_t stage_land_rows() { return (uint32_t)stage_bytes(D) - 16 * kR
 // Merge the n pieces of a split unit with the log-sum-exp identity,
 // LSE = ln sum_i exp(lse_i) and O = sum_i exp(lse_i - LSE) O_i, in two
 // passes.  The pieces' partial rows and LSEs are brought into a landing zone
-// (`land`, with `land_rows` bytes for rows and the LSEs after them) with
-// bulk loads, up to 16 pieces' rows at a time; the LSEs of all pieces come
-// with the first landing when there are at most 16 pieces (else each batch
-// brings its own and the row statistics read them from global memory).
+// (`land`, with `land_rows` bytes for rows and then `lse_slots` pieces'
+// LSEs) with bulk loads, as many pieces' rows at a time as fit; the LSEs of
+// all pieces come with the first landing when there are at most `lse_slots`
+// pieces (else each batch brings its own and the row statistics read them
+// from global memory).
 // First the row statistics, spread over a power-of-two group of lanes per
 // row and reduced with a running maximum; then every lane accumulates its
 // D / 32 columns of every row with the weights known up front, so the
@@ -788,14 +794,14 @@ constexpr uint32_t stage_land_rows() { return (uint32_t)stage_bytes(D) - 16 * kR
 template <int D, bool kBf16>
 __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int rows, int unit, int lane,
                              uint8_t *smem, uint32_t ostage, uint32_t land, uint32_t land_rows,
-                             uint32_t mbar, uint32_t &mk, int own) {
+                             uint32_t mbar, uint32_t &mk, int own, int lse_slots) {
   constexpr int VEC = D / 32;
   constexpr float kLog2e = 1.4426950408889634f;
   const int n = sg.n_pieces, cf = sg.c_first;
   auto slot_of = [&](int i) -> size_t { return i == 0 ? (size_t)cf * 2 + 1 : (size_t)(cf + i) * 2; };
   const uint32_t pbytes = (uint32_t)rows * D * 4;
-  const int cap = min(kRowsPerTile, (int)(land_rows / pbytes));
-  const bool all_lse = n <= kRowsPerTile;  // every piece's LSEs come with the first landing
+  const int cap = min(lse_slots, (int)(land_rows / pbytes));
+  const bool all_lse = n <= lse_slots;  // every piece's LSEs come with the first landing
   auto issue = [&](int i0, int k) {  // bulk loads of pieces i0 .. i0 + k - 1
     fence_proxy_async_smem();  // earlier reads of the landing zone precede the new loads
     __syncwarp();
@@ -1037,14 +1043,18 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
     // A split unit's landing zone: the staging buffer when all its pieces'
     // rows fit there, else the ring stage this job came in (kept until the
     // piece has been counted, and merged if it was the last).
-    const bool hold = sg.kind != 0 && (uint32_t)sg.n_pieces * rows * D * 4 > (uint32_t)kLandRows;
-    const uint32_t land = hold ? sbase : oland;
-    const uint32_t land_rows = hold ? stage_land_rows<D>() : (uint32_t)kLandRows;
+    // The CTA's last segment lands a merge in the whole ring, which nothing
+    // loads into any more.
+    const bool hold = sg.kind != 0 && !sg.last && (uint32_t)sg.n_pieces * rows * D * 4 > (uint32_t)kLandRows;
+    const uint32_t land = sg.last ? ring : hold ? sbase : oland;
+    const uint32_t land_rows = sg.last ? kStages * 2 * KV_BYTES - kRingLseSlots * kRowsPerTile * 4
+                               : hold ? stage_land_rows<D>() : (uint32_t)kLandRows;
+    const int lse_slots = sg.last ? kRingLseSlots : kRowsPerTile;
     const int own = (int)blockIdx.x - sg.c_first;  // this piece's index in the unit
     seen = __shfl_sync(0xffffffffu, seen, 0);
     const bool merge_now = sg.kind != 0 && (seen >> 32) == (unsigned long long)a.epoch &&
                            (int)(seen & 0xffffffffull) == sg.n_pieces - 1 &&
-                           sg.n_pieces <= min(kRowsPerTile, (int)(land_rows / ((uint32_t)rows * D * 4)));
+                           sg.n_pieces <= min(lse_slots, (int)(land_rows / ((uint32_t)rows * D * 4)));
     __syncwarp();  // every lane has read the stage before it may become the landing zone
     const uint32_t dst_rows = merge_now ? land + (uint32_t)own * rows * D * 4 : ostage;
 #pragma unroll
@@ -1098,7 +1108,8 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
       // fenced first); the acquire lets the last piece read everyone's.
       bool ok = true;
       if (merge_now) {
-        ok = merge_pieces<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, merge_bar, mk, own);
+        ok = merge_pieces<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, merge_bar, mk, own,
+                                    lse_slots);
       } else {
         unsigned long long old = 0;
         if (lane == 0) {
@@ -1108,7 +1119,8 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
         }
         old = __shfl_sync(0xffffffffu, old, 0);
         if ((int)(old & 0xffffffffull) + 1 == sg.n_pieces)
-          ok = merge_pieces<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, merge_bar, mk, -1);
+          ok = merge_pieces<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, merge_bar, mk, -1,
+                                      lse_slots);
       }
       if (hold) {
         fence_proxy_async_smem();  // reads of the landing zone precede the stage's next TMA loads
