@@ -129,6 +129,7 @@ mxa_status_t mxa_plan(const mxa_decode_params_t *p, int num_splits, int sm_count
   const int RT = (p->q_len * G + kRowsPerTile - 1) / kRowsPerTile;
   const long long units = (long long)p->B * p->Hkv * RT;
   const int T = block_tokens(p->D);
+  const int rows = p->q_len * G < kRowsPerTile ? p->q_len * G : kRowsPerTile;  // packed rows of a full tile
   if (num_splits > 0) {
     if (units * num_splits > INT32_MAX) return MXA_ERR_UNSUPPORTED;
     out.schedule = MXA_SCHED_UNIFORM;
@@ -146,7 +147,7 @@ mxa_status_t mxa_plan(const mxa_decode_params_t *p, int num_splits, int sm_count
       long long cap = units * (max_blocks + 3) / 4;
       if (cap < 1) cap = 1;
       out.schedule = MXA_SCHED_BALANCED;
-      out.unit_cost = kUnitCost;
+      out.unit_cost = unit_cost_for_rows(rows);
       out.grid = (int)(slots < cap ? slots : cap);
       out.num_splits = units > 0 ? (int)ceil_div_ll(out.grid, units) : 1;
     } else {
@@ -178,7 +179,6 @@ mxa_status_t mxa_plan_balanced(const mxa_decode_params_t *p, int grid, int sm_co
   if (st != MXA_OK) return st;
   if (p->B > kMaxBalancedRows) return MXA_ERR_UNSUPPORTED;
   out.schedule = MXA_SCHED_BALANCED;
-  out.unit_cost = kUnitCost;
   out.grid = grid;
   out.num_splits = out.units > 0 ? (grid + out.units - 1) / out.units : 1;
   finish_plan(p, &out);

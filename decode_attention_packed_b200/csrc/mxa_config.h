@@ -16,8 +16,13 @@ constexpr int kSmemPerSm = 228 * 1024;                  // B200 shared memory pe
 constexpr int kSmemReservedPerCta = 1024;               // driver-reserved shared memory per CTA
 constexpr int kMaxThreadsPerSm = 2048;
 constexpr int kMaxBalancedRows = 12288;                 // balanced schedule scans B rows in smem
-constexpr int kUnitCost = 2;                            // fixed cost of a unit, in KV blocks
 constexpr int kMaxUnitCost = 64;
+
+// Fixed cost of a unit in the balanced schedule, in KV blocks: the work a
+// unit needs besides streaming its keys (the cross-warp merge, the output
+// staging and stores, the arrival and merge of a split unit) grows with its
+// packed query rows, and measures at about one block per two rows on B200.
+constexpr int unit_cost_for_rows(int rows) { return rows > 2 ? (rows + 1) / 2 : 1; }
 
 // KV tokens per pipeline stage: every stage carries T x D elements of K and
 // of V (16 KiB each in 16-bit types), so T = 8192 / D.  Three stages per CTA

@@ -1040,21 +1040,25 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
         }
       }
     }
-    // A split unit's landing zone: the staging buffer when all its pieces'
-    // rows fit there, else the ring stage this job came in (kept until the
-    // piece has been counted, and merged if it was the last).
-    // The CTA's last segment lands a merge in the whole ring, which nothing
-    // loads into any more.
-    const bool hold = sg.kind != 0 && !sg.last && (uint32_t)sg.n_pieces * rows * D * 4 > (uint32_t)kLandRows;
+    // A split unit's landing zone.  The CTA's last segment uses the whole
+    // ring, which nothing loads into any more.  Otherwise a piece that will
+    // merge at once (every other piece has arrived) and whose unit's rows
+    // do not fit the staging buffer keeps the ring stage this job came in
+    // for the merge; all other pieces give the stage straight back, so the
+    // ring stays full, and a piece that turns out to be the last to arrive
+    // merges through the staging buffer, in as many landings as needed.
+    seen = __shfl_sync(0xffffffffu, seen, 0);
+    const uint32_t pbytes = (uint32_t)rows * D * 4;
+    const bool all_here = sg.kind != 0 && (seen >> 32) == (unsigned long long)a.epoch &&
+                          (int)(seen & 0xffffffffull) == sg.n_pieces - 1;
+    const bool hold = all_here && !sg.last && (uint32_t)sg.n_pieces * pbytes > (uint32_t)kLandRows &&
+                      sg.n_pieces <= min(kRowsPerTile, (int)(stage_land_rows<D>() / pbytes));
     const uint32_t land = sg.last ? ring : hold ? sbase : oland;
     const uint32_t land_rows = sg.last ? kStages * 2 * KV_BYTES - kRingLseSlots * kRowsPerTile * 4
                                : hold ? stage_land_rows<D>() : (uint32_t)kLandRows;
     const int lse_slots = sg.last ? kRingLseSlots : kRowsPerTile;
     const int own = (int)blockIdx.x - sg.c_first;  // this piece's index in the unit
-    seen = __shfl_sync(0xffffffffu, seen, 0);
-    const bool merge_now = sg.kind != 0 && (seen >> 32) == (unsigned long long)a.epoch &&
-                           (int)(seen & 0xffffffffull) == sg.n_pieces - 1 &&
-                           sg.n_pieces <= min(lse_slots, (int)(land_rows / ((uint32_t)rows * D * 4)));
+    const bool merge_now = all_here && sg.n_pieces <= min(lse_slots, (int)(land_rows / pbytes));
     __syncwarp();  // every lane has read the stage before it may become the landing zone
     const uint32_t dst_rows = merge_now ? land + (uint32_t)own * rows * D * 4 : ostage;
 #pragma unroll
