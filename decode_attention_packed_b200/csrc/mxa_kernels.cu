@@ -32,6 +32,8 @@
 //    RightDownCausal mask for the draft tokens of a speculative step; 源码级
 //    原理: a balanced division of the KV work over the cores, with a reduce
 //    for rows whose keys span several cores.
+#include <type_traits>
+
 #include "mxa_config.h"
 #include "mxa_device.cuh"
 #include "mxa_launch.h"
@@ -791,7 +793,7 @@ constexpr uint32_t stage_land_rows() { return (uint32_t)stage_bytes(D) - 16 * kR
 // count).  `own` >= 0 names a piece the caller has already placed in the
 // landing zone (rows and LSEs at its index; then all n pieces fit one
 // landing).  Returns false if a bounded wait ran out.
-template <int D, bool kBf16>
+template <int D, bool kBf16, int NR>
 __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int rows, int unit, int lane,
                              uint8_t *smem, uint32_t ostage, uint32_t land, uint32_t land_rows,
                              uint32_t mbar, uint32_t &mk, int own, int lse_slots) {
@@ -865,17 +867,17 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
     const int mrow = sg.rt * kRowsPerTile + r1, t = mrow / a.G, g = mrow % a.G;
     a.lse[((size_t)sg.b * a.Hq + (size_t)sg.h * a.G + g) * a.q_len + t] = lse2 * kLn2;
   }
-  float row_lse[kRowsPerTile];
+  float row_lse[NR];
 #pragma unroll
-  for (int rr = 0; rr < kRowsPerTile; ++rr) row_lse[rr] = __shfl_sync(0xffffffffu, lse2, (rr * lpr) & 31);
+  for (int rr = 0; rr < NR; ++rr) row_lse[rr] = __shfl_sync(0xffffffffu, lse2, (rr * lpr) & 31);
 
   // ---- pass 2: O = sum_i w_i O_i with w_i = exp(lse_i - LSE) ----
-  // All 16 row slots are computed without branches so the loads overlap;
-  // slots past `rows` read a valid row and their sums are never stored.
+  // All NR row slots (NR >= rows) are computed without branches so the
+  // loads overlap; slots past `rows` read a valid row and are never stored.
   const int col = lane * VEC;
-  float acc[kRowsPerTile][VEC];
+  float acc[NR][VEC];
 #pragma unroll
-  for (int rr = 0; rr < kRowsPerTile; ++rr)
+  for (int rr = 0; rr < NR; ++rr)
 #pragma unroll
     for (int v = 0; v < VEC; ++v) acc[rr][v] = 0.f;
   for (int i0 = 0; i0 < n; i0 += cap) {
@@ -885,7 +887,7 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
       const float *lp = land_l + (all_lse ? i0 + p : p) * kRowsPerTile;
       const float *op = land_o + p * rows * D + col;
 #pragma unroll
-      for (int rr = 0; rr < kRowsPerTile; ++rr) {
+      for (int rr = 0; rr < NR; ++rr) {
         const int rc = rr < rows ? rr : rows - 1;
         const float l = lp[rr] * kLog2e;
         const float w = l == -INFINITY ? 0.f : ex2(l - row_lse[rr]);
@@ -902,7 +904,7 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
   }
   __syncwarp();  // every lane is done with the landing zone, which may be the staging buffer
 #pragma unroll
-  for (int rr = 0; rr < kRowsPerTile; ++rr)
+  for (int rr = 0; rr < NR; ++rr)
     if (rr < rows) stage_out_vec<D, kBf16>(smem, ostage, rr, col, acc[rr]);
   fence_proxy_async_smem();  // staged rows are read by the bulk stores
   __syncwarp();
@@ -912,6 +914,21 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
     a.counters[unit] = 0ull;  // every piece has arrived; leave it clean
   }
   return true;
+}
+
+// merge_pieces for the smallest power-of-two row count (2 to 16) >= rows.
+template <int D, bool kBf16>
+__device__ __forceinline__ bool merge_unit(const DecodeArgs &a, const SegmentDesc &sg, int rows, int unit,
+                                           int lane, uint8_t *smem, uint32_t ostage, uint32_t land,
+                                           uint32_t land_rows, uint32_t mbar, uint32_t &mk, int own,
+                                           int lse_slots) {
+  if (rows <= 2)
+    return merge_pieces<D, kBf16, 2>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, mbar, mk, own, lse_slots);
+  if (rows <= 4)
+    return merge_pieces<D, kBf16, 4>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, mbar, mk, own, lse_slots);
+  if (rows <= 8)
+    return merge_pieces<D, kBf16, 8>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, mbar, mk, own, lse_slots);
+  return merge_pieces<D, kBf16, 16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, mbar, mk, own, lse_slots);
 }
 
 template <int D, bool kBf16>
@@ -1017,65 +1034,78 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
     }
     // O of each row: the four warps' unnormalised partials, weighted.  A
     // warp whose weight is 0 left zeros (or finite values) in its slice, so
-    // every load is made.  All 16 row slots are loaded before anything is
-    // staged and without branches, so the loads overlap; slots past `rows`
-    // read a valid row and are never stored.
+    // every load is made.  The NR row slots (the smallest power of two from
+    // 2 to 16 that holds `rows`) are loaded before anything is staged and
+    // without branches, so the loads overlap; slots past `rows` read a valid
+    // row and are never stored.
+    //
+    // A split unit's landing zone is chosen meanwhile.  The CTA's last
+    // segment uses the whole ring, which nothing loads into any more.
+    // Otherwise a piece that will merge at once (every other piece has
+    // arrived) and whose unit's rows do not fit the staging buffer keeps the
+    // ring stage this job came in for the merge; all other pieces give the
+    // stage straight back, so the ring stays full, and a piece that turns
+    // out to be the last to arrive merges through the staging buffer, in as
+    // many landings as needed.
     const float *hbase = reinterpret_cast<const float *>(smem + (sbase - smem_addr(smem)));
-    float acc[kRowsPerTile][VEC];
-#pragma unroll
-    for (int rr = 0; rr < kRowsPerTile; ++rr) {
-      const int rc = rr < rows ? rr : rows - 1;
-#pragma unroll
-      for (int v = 0; v < VEC; ++v) acc[rr][v] = 0.f;
-#pragma unroll
-      for (int w = 0; w < kMathWarps; ++w) {
-        const float wg = __shfl_sync(0xffffffffu, wgt[w], rr);
-        const float *src = hbase + (handoff_addr<D>(sbase, w, rc, col) - sbase) / 4;
-        if constexpr (VEC == 4) {
-          const float4 v = *reinterpret_cast<const float4 *>(src);
-          acc[rr][0] += wg * v.x; acc[rr][1] += wg * v.y; acc[rr][2] += wg * v.z; acc[rr][3] += wg * v.w;
-        } else {
-          const float2 v = *reinterpret_cast<const float2 *>(src);
-          acc[rr][0] += wg * v.x; acc[rr][1] += wg * v.y;
-        }
-      }
-    }
-    // A split unit's landing zone.  The CTA's last segment uses the whole
-    // ring, which nothing loads into any more.  Otherwise a piece that will
-    // merge at once (every other piece has arrived) and whose unit's rows
-    // do not fit the staging buffer keeps the ring stage this job came in
-    // for the merge; all other pieces give the stage straight back, so the
-    // ring stays full, and a piece that turns out to be the last to arrive
-    // merges through the staging buffer, in as many landings as needed.
-    seen = __shfl_sync(0xffffffffu, seen, 0);
     const uint32_t pbytes = (uint32_t)rows * D * 4;
-    const bool all_here = sg.kind != 0 && (seen >> 32) == (unsigned long long)a.epoch &&
-                          (int)(seen & 0xffffffffull) == sg.n_pieces - 1;
-    const bool hold = all_here && !sg.last && (uint32_t)sg.n_pieces * pbytes > (uint32_t)kLandRows &&
-                      sg.n_pieces <= min(kRowsPerTile, (int)(stage_land_rows<D>() / pbytes));
-    const uint32_t land = sg.last ? ring : hold ? sbase : oland;
-    const uint32_t land_rows = sg.last ? kStages * 2 * KV_BYTES - kRingLseSlots * kRowsPerTile * 4
-                               : hold ? stage_land_rows<D>() : (uint32_t)kLandRows;
-    const int lse_slots = sg.last ? kRingLseSlots : kRowsPerTile;
     const int own = (int)blockIdx.x - sg.c_first;  // this piece's index in the unit
-    const bool merge_now = all_here && sg.n_pieces <= min(lse_slots, (int)(land_rows / pbytes));
-    __syncwarp();  // every lane has read the stage before it may become the landing zone
-    const uint32_t dst_rows = merge_now ? land + (uint32_t)own * rows * D * 4 : ostage;
+    bool hold = false, merge_now = false;
+    uint32_t land = oland, land_rows = (uint32_t)kLandRows, dst_rows = ostage;
+    int lse_slots = kRowsPerTile;
+    auto merge_warps = [&](auto row_slots) {
+      constexpr int NR = decltype(row_slots)::value;
+      float acc[NR][VEC];
 #pragma unroll
-    for (int rr = 0; rr < kRowsPerTile; ++rr) {
-      if (rr < rows) {
-        if (sg.kind == 0) {
-          stage_out_vec<D, kBf16>(smem, ostage, rr, col, acc[rr]);
-        } else {  // fp32 partial rows, pitch D * 4 bytes
-          float *dst = reinterpret_cast<float *>(smem + (dst_rows - smem_addr(smem))) + rr * D + col;
+      for (int rr = 0; rr < NR; ++rr) {
+        const int rc = rr < rows ? rr : rows - 1;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[rr][v] = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMathWarps; ++w) {
+          const float wg = __shfl_sync(0xffffffffu, wgt[w], rr);
+          const float *src = hbase + (handoff_addr<D>(sbase, w, rc, col) - sbase) / 4;
           if constexpr (VEC == 4) {
-            *reinterpret_cast<float4 *>(dst) = make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
+            const float4 v = *reinterpret_cast<const float4 *>(src);
+            acc[rr][0] += wg * v.x; acc[rr][1] += wg * v.y; acc[rr][2] += wg * v.z; acc[rr][3] += wg * v.w;
           } else {
-            *reinterpret_cast<float2 *>(dst) = make_float2(acc[rr][0], acc[rr][1]);
+            const float2 v = *reinterpret_cast<const float2 *>(src);
+            acc[rr][0] += wg * v.x; acc[rr][1] += wg * v.y;
           }
         }
       }
-    }
+      seen = __shfl_sync(0xffffffffu, seen, 0);
+      const bool all_here = sg.kind != 0 && (seen >> 32) == (unsigned long long)a.epoch &&
+                            (int)(seen & 0xffffffffull) == sg.n_pieces - 1;
+      hold = all_here && !sg.last && (uint32_t)sg.n_pieces * pbytes > (uint32_t)kLandRows &&
+             sg.n_pieces <= min(kRowsPerTile, (int)(stage_land_rows<D>() / pbytes));
+      land = sg.last ? ring : hold ? sbase : oland;
+      land_rows = sg.last ? kStages * 2 * KV_BYTES - kRingLseSlots * kRowsPerTile * 4
+                  : hold ? stage_land_rows<D>() : (uint32_t)kLandRows;
+      lse_slots = sg.last ? kRingLseSlots : kRowsPerTile;
+      merge_now = all_here && sg.n_pieces <= min(lse_slots, (int)(land_rows / pbytes));
+      __syncwarp();  // every lane has read the stage before it may become the landing zone
+      dst_rows = merge_now ? land + (uint32_t)own * pbytes : ostage;
+#pragma unroll
+      for (int rr = 0; rr < NR; ++rr) {
+        if (rr < rows) {
+          if (sg.kind == 0) {
+            stage_out_vec<D, kBf16>(smem, ostage, rr, col, acc[rr]);
+          } else {  // fp32 partial rows, pitch D * 4 bytes
+            float *dst = reinterpret_cast<float *>(smem + (dst_rows - smem_addr(smem))) + rr * D + col;
+            if constexpr (VEC == 4) {
+              *reinterpret_cast<float4 *>(dst) = make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
+            } else {
+              *reinterpret_cast<float2 *>(dst) = make_float2(acc[rr][0], acc[rr][1]);
+            }
+          }
+        }
+      }
+    };
+    if (rows <= 2) merge_warps(std::integral_constant<int, 2>{});
+    else if (rows <= 4) merge_warps(std::integral_constant<int, 4>{});
+    else if (rows <= 8) merge_warps(std::integral_constant<int, 8>{});
+    else merge_warps(std::integral_constant<int, 16>{});
     // row statistics: lane r < rows owns row r
     if (lane < rows) {
       if (sg.kind == 0) {
@@ -1112,7 +1142,7 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
       // fenced first); the acquire lets the last piece read everyone's.
       bool ok = true;
       if (merge_now) {
-        ok = merge_pieces<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, merge_bar, mk, own,
+        ok = merge_unit<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, merge_bar, mk, own,
                                     lse_slots);
       } else {
         unsigned long long old = 0;
@@ -1123,7 +1153,7 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
         }
         old = __shfl_sync(0xffffffffu, old, 0);
         if ((int)(old & 0xffffffffull) + 1 == sg.n_pieces)
-          ok = merge_pieces<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, merge_bar, mk, -1,
+          ok = merge_unit<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, merge_bar, mk, -1,
                                       lse_slots);
       }
       if (hold) {
