@@ -807,17 +807,22 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
   auto issue = [&](int i0, int k) {  // bulk loads of pieces i0 .. i0 + k - 1
     fence_proxy_async_smem();  // earlier reads of the landing zone precede the new loads
     __syncwarp();
+    const int l0 = all_lse ? 0 : i0, nl = all_lse ? (i0 == 0 ? n : 0) : k;
     if (lane == 0) {
-      const int l0 = all_lse ? 0 : i0, nl = all_lse ? (i0 == 0 ? n : 0) : k;
       const int ko = (own >= i0 && own < i0 + k) ? 1 : 0, lo = (own >= l0 && own < l0 + nl) ? 1 : 0;
       mbar_arrive_expect_tx(mbar, (uint32_t)(k - ko) * pbytes + (uint32_t)(nl - lo) * kRowsPerTile * 4);
-      for (int p = 0; p < k; ++p)
-        if (i0 + p != own)
-          bulk_load(land + (uint32_t)p * pbytes, a.o_part + slot_of(i0 + p) * kRowsPerTile * D, pbytes, mbar);
-      for (int p = 0; p < nl; ++p)
-        if (l0 + p != own)
-          bulk_load(land + land_rows + (uint32_t)p * kRowsPerTile * 4, a.lse_part + slot_of(l0 + p) * kRowsPerTile,
-                    kRowsPerTile * 4, mbar);
+    }
+    __syncwarp();
+    // the lanes issue the copies together: rows of pieces first, then LSEs
+    for (int c = lane; c < k + nl; c += 32) {
+      if (c < k) {
+        if (i0 + c != own)
+          bulk_load(land + (uint32_t)c * pbytes, a.o_part + slot_of(i0 + c) * kRowsPerTile * D, pbytes, mbar);
+      } else if (l0 + c - k != own) {
+        const int p = c - k;
+        bulk_load(land + land_rows + (uint32_t)p * kRowsPerTile * 4, a.lse_part + slot_of(l0 + p) * kRowsPerTile,
+                  kRowsPerTile * 4, mbar);
+      }
     }
     __syncwarp();
   };
@@ -867,6 +872,16 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
     const int mrow = sg.rt * kRowsPerTile + r1, t = mrow / a.G, g = mrow % a.G;
     a.lse[((size_t)sg.b * a.Hq + (size_t)sg.h * a.G + g) * a.q_len + t] = lse2 * kLn2;
   }
+  // With every LSE landed, the lanes that read a piece's LSE turn it into
+  // its weight exp(lse_i - LSE) in place, once for all lanes.
+  if (all_lse && r1 < rows) {
+    float *lw = const_cast<float *>(land_l);
+    for (int p = j1; p < n; p += lpr) {
+      const float l = lw[p * kRowsPerTile + r1] * kLog2e;
+      lw[p * kRowsPerTile + r1] = (l == -INFINITY || lse2 == -INFINITY) ? 0.f : ex2(l - lse2);
+    }
+  }
+  __syncwarp();
   float row_lse[NR];
 #pragma unroll
   for (int rr = 0; rr < NR; ++rr) row_lse[rr] = __shfl_sync(0xffffffffu, lse2, (rr * lpr) & 31);
@@ -889,8 +904,13 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
 #pragma unroll
       for (int rr = 0; rr < NR; ++rr) {
         const int rc = rr < rows ? rr : rows - 1;
-        const float l = lp[rr] * kLog2e;
-        const float w = l == -INFINITY ? 0.f : ex2(l - row_lse[rr]);
+        float w;
+        if (all_lse) {
+          w = lp[rr];  // already the weight
+        } else {
+          const float l = lp[rr] * kLog2e;
+          w = l == -INFINITY ? 0.f : ex2(l - row_lse[rr]);
+        }
         if constexpr (VEC == 4) {
           const float4 v = *reinterpret_cast<const float4 *>(op + rc * D);
           acc[rr][0] += w * v.x; acc[rr][1] += w * v.y; acc[rr][2] += w * v.z; acc[rr][3] += w * v.w;
