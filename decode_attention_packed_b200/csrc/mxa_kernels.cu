@@ -279,6 +279,10 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
   const int bt = a.box_tokens;
   const int ps = a.page_size;
   const uint16_t *q = reinterpret_cast<const uint16_t *>(a.q);
+  // The KV cache is read once per call: its lines leave L2 first, so the
+  // lengths, block table, queries and split partials that every call
+  // touches stay there.
+  const uint64_t kv_policy = l2_policy_evict_first();
 
   if (lane == 0) {
     prefetch_tmap(&tm.k);
@@ -395,8 +399,8 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
             const int row = a.contiguous ? seg.b * ps + tok : page * ps + tok % ps;
             const uint32_t dst = ring + (uint32_t)s * (2 * KV_BYTES) + (uint32_t)kv * KV_BYTES +
                                  (uint32_t)ch * (T * 128) + (uint32_t)(box * bt) * 128;
-            tma_load_3d(dst, kv ? (const void *)&tm.v : (const void *)&tm.k, ch * 64, seg.h, row,
-                        bar_addr(smem, D, B_FULL(s)));
+            tma_load_3d_hint(dst, kv ? (const void *)&tm.v : (const void *)&tm.k, ch * 64, seg.h, row,
+                        bar_addr(smem, D, B_FULL(s)), kv_policy);
           }
         }
         ++it;
