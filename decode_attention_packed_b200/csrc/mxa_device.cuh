@@ -143,17 +143,8 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
-// 3-D tiled TMA load global -> shared, completing on `bar` (tx bytes).
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int x, int y, int z,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-
-// As tma_load_3d, with an L2 cache policy (from l2_policy_evict_first).
+// 3-D tiled TMA load global -> shared, completing on `bar` (tx bytes), with
+// an L2 cache policy (from l2_policy_evict_first).
 __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const void *tmap, int x, int y, int z,
                                                  uint32_t bar, uint64_t policy) {
   asm volatile(

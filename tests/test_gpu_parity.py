@@ -133,6 +133,23 @@ def test_balanced_unit_costs_edge_lengths(unit_cost):
     check(inp, out, lse)
 
 
+@pytest.mark.parametrize("D,dtype,G", [(128, "bf16", 16), (64, "f16", 1), (128, "f16", 3)])
+@pytest.mark.parametrize("grid", [40, 130])
+def test_one_unit_in_many_pieces(D, dtype, G, grid):
+    # a single long row cut into more pieces than one landing's LSE slots
+    # hold: the merge lands its pieces in several batches and takes the row
+    # statistics from global memory
+    w = Workload(name="many", B=1, q_len=1, Hq=G, Hkv=1, D=D, dtype=dtype, page_size=64, causal=False,
+                 lengths="const:16000", seed=77)
+    inp = make_inputs(w)
+    dev = to_dev(inp)
+    q, k, v, bt, sl = dev
+    plan = mxa.mxa_plan_balanced(mxa.params_for(q, k, bt, inp.max_seqlen_k), grid)
+    assert plan.needs_combine == 1
+    out, lse, _ = run_gpu(inp, plan=plan, dev=dev)
+    check(inp, out, lse)
+
+
 # --------------------------------------------------------------------------
 # shapes and edges at sizes the oracle finishes in seconds
 # --------------------------------------------------------------------------
