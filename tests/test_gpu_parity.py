@@ -150,6 +150,18 @@ def test_one_unit_in_many_pieces(D, dtype, G, grid):
     check(inp, out, lse)
 
 
+@pytest.mark.parametrize("B", [12288, 12289])
+def test_row_limit_of_the_balanced_schedule(B):
+    # the largest batch the balanced prologue scans, and one row more (the
+    # automatic plan then uses the uniform schedule)
+    w = Workload(name="rows", B=B, q_len=1, Hq=2, Hkv=1, D=64, dtype="f16", page_size=16, causal=False,
+                 lengths="uniform:0:64", seed=90)
+    inp = make_inputs(w)
+    out, lse, plan = run_gpu(inp)
+    assert plan.schedule == (mxa.MXA_SCHED_BALANCED if B <= 12288 else mxa.MXA_SCHED_UNIFORM)
+    check(inp, out, lse)
+
+
 # --------------------------------------------------------------------------
 # shapes and edges at sizes the oracle finishes in seconds
 # --------------------------------------------------------------------------

@@ -130,6 +130,20 @@ def test_plan_uniform_and_row_tiles():
     assert mxa.mxa_plan(params(D=64), 1, sm_count=148).block_tokens == 128
 
 
+def test_plan_switches_to_uniform_past_the_balanced_row_limit():
+    # the balanced prologue scans at most 12288 rows in shared memory; past
+    # that the automatic plan uses the page's num_splits rule (uniform)
+    at = mxa.mxa_plan(params(B=12288, max_seqlen_k=256, max_pages_per_seq=4, num_pages=50000), 0,
+                      sm_count=148)
+    past = mxa.mxa_plan(params(B=12289, max_seqlen_k=256, max_pages_per_seq=4, num_pages=50000), 0,
+                        sm_count=148)
+    assert at.schedule == MXA_SCHED_BALANCED
+    assert past.schedule == MXA_SCHED_UNIFORM and past.num_splits == 1  # 98k units fill the GPU
+    p = mxa_plan_t()
+    pp = params(B=12289, max_seqlen_k=256, max_pages_per_seq=4, num_pages=50000)
+    assert mxa._lib.mxa_plan_balanced(ctypes.byref(pp), 296, 148, ctypes.byref(p)) == MXA_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(D=96), MXA_ERR_UNSUPPORTED),
     (dict(D=256), MXA_ERR_UNSUPPORTED),
