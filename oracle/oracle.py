@@ -81,6 +81,37 @@ def decode(q, k_cache, v_cache, block_table, cache_seqlens, *, Hkv: int,
     return out, lse
 
 
+def append_kv(k_cache, v_cache, k_new, v_new, block_table, cache_seqlens, *, page_size: int):
+    """Write each row's new tokens into copies of the caches; return the copies.
+
+    The new keys and values that a decode call appends before attending
+    ("Flash-Attention GQA 性能调优: pack_gqa 与 num_splits", the k / v arguments
+    of flash_attn_with_kvcache next to cache_seqlens; "MXFlashAttn 1.4.0",
+    能力矩阵: paged KV append).  Row b's new token t goes to logical position
+    L_b + t of the row (L_b = cache_seqlens[b]): page
+    block_table[b, (L_b + t) // page_size], slot (L_b + t) % page_size, or
+    row b, slot L_b + t of a contiguous cache (block_table None).  The
+    values are copied bit for bit.
+
+    k_cache/v_cache as for decode(); k_new/v_new [B, q_len, Hkv, D].
+    """
+    kb, vb = _bits(k_cache).copy(), _bits(v_cache).copy()
+    knb, vnb = _bits(k_new), _bits(v_new)
+    B, q_len = knb.shape[0], knb.shape[1]
+    L = np.asarray(cache_seqlens, dtype=np.int64)
+    bt = None if block_table is None else np.asarray(block_table, dtype=np.int64)
+    for b in range(B):
+        for t in range(q_len):
+            pos = int(L[b]) + t
+            if bt is None:
+                page, slot = b, pos
+            else:
+                page, slot = int(bt[b, pos // page_size]), pos % page_size
+            kb[page, slot] = knb[b, t]
+            vb[page, slot] = vnb[b, t]
+    return kb, vb
+
+
 def combine(o_part: np.ndarray, lse_part: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
     """Exact LSE merge.  o_part [S, rows, D], lse_part [S, rows] (float64)."""
     lib = _load()

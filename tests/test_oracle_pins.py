@@ -316,3 +316,77 @@ def test_brute_force_tiny(seed):
     fin = np.isfinite(bl)
     assert (np.isfinite(l) == fin).all()
     np.testing.assert_allclose(l[fin], bl[fin], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# appending new tokens to the cache (k / v of flash_attn_with_kvcache)
+# --------------------------------------------------------------------------
+
+def _labelled(shape, base):
+    """bf16 tensor whose element values (small integers, exact in bf16) name their index."""
+    idx = np.arange(int(np.prod(shape)), dtype=np.float32).reshape(shape) % 251 + base
+    return torch.from_numpy(idx).to(torch.bfloat16)
+
+
+def test_append_writes_each_token_to_its_page_and_slot():
+    # two rows, pages of 4 slots; row 0 holds 2 keys, row 1 holds 5; 3 new tokens each
+    bt = np.array([[3, 0], [1, 2]], dtype=np.int32)
+    L = np.array([2, 5], dtype=np.int32)
+    k_cache = torch.zeros((4, 4, 1, 2), dtype=torch.bfloat16)
+    v_cache = torch.zeros((4, 4, 1, 2), dtype=torch.bfloat16)
+    k_new = _labelled((2, 3, 1, 2), 1.0)
+    v_new = _labelled((2, 3, 1, 2), 300.0)
+    kb, vb = oracle.append_kv(k_cache, v_cache, k_new, v_new, bt, L, page_size=4)
+    kf = torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16).float()
+    vf = torch.from_numpy(vb.view(np.int16)).view(torch.bfloat16).float()
+    # written by hand: (row, new token) -> (page, slot)
+    where = {(0, 0): (3, 2), (0, 1): (3, 3), (0, 2): (0, 0),
+             (1, 0): (2, 1), (1, 1): (2, 2), (1, 2): (2, 3)}
+    written = set()
+    for (b, t), (page, slot) in where.items():
+        assert torch.equal(kf[page, slot], k_new[b, t].float())
+        assert torch.equal(vf[page, slot], v_new[b, t].float())
+        written.add((page, slot))
+    for page in range(4):
+        for slot in range(4):
+            if (page, slot) not in written:
+                assert not kf[page, slot].any() and not vf[page, slot].any()
+
+
+def test_append_then_decode_equals_decoding_the_full_cache():
+    # a cache that already holds L + q_len keys per row, and the same cache
+    # with its last q_len keys per row blanked and handed over as new tokens
+    q_len = 3
+    w = wl(B=3, q_len=q_len, Hq=8, Hkv=2, D=32, page_size=4, lengths="list:7,9,12", causal=True)
+    full = make_inputs(w)
+    L_before = full.cache_seqlens.numpy() - q_len
+    k_new = torch.zeros((w.B, q_len, w.Hkv, w.D), dtype=full.k_cache.dtype)
+    v_new = torch.zeros_like(k_new)
+    k_blank, v_blank = full.k_cache.clone(), full.v_cache.clone()
+    for b in range(w.B):
+        for t in range(q_len):
+            pos = int(L_before[b]) + t
+            page, slot = int(full.block_table[b, pos // 4]), pos % 4
+            k_new[b, t], v_new[b, t] = full.k_cache[page, slot], full.v_cache[page, slot]
+            k_blank[page, slot] = 0
+            v_blank[page, slot] = 0
+    kb, vb = oracle.append_kv(k_blank, v_blank, k_new, v_new, full.block_table, L_before, page_size=4)
+    assert np.array_equal(kb, oracle.oracle._bits(full.k_cache))
+    assert np.array_equal(vb, oracle.oracle._bits(full.v_cache))
+    ref_o, ref_l = run_oracle(full)
+    got_o, got_l = oracle.decode(full.q, kb, vb, full.block_table, full.cache_seqlens, Hkv=w.Hkv,
+                                 page_size=4, dtype=w.dtype, scale=w.scale, causal=True)
+    assert np.array_equal(got_o, ref_o) and np.array_equal(got_l, ref_l)
+
+
+def test_append_to_a_contiguous_cache():
+    k_cache = torch.zeros((2, 8, 1, 2), dtype=torch.bfloat16)
+    v_cache = torch.zeros_like(k_cache)
+    k_new = _labelled((2, 2, 1, 2), 5.0)
+    v_new = _labelled((2, 2, 1, 2), 77.0)
+    kb, vb = oracle.append_kv(k_cache, v_cache, k_new, v_new, None, np.array([0, 6], dtype=np.int32),
+                              page_size=8)
+    kf = torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16)
+    assert torch.equal(kf[0, 0], k_new[0, 0]) and torch.equal(kf[0, 1], k_new[0, 1])
+    assert torch.equal(kf[1, 6], k_new[1, 0]) and torch.equal(kf[1, 7], k_new[1, 1])
+    assert int((kf != 0).sum()) == int((k_new != 0).sum())
