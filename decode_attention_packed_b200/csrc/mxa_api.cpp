@@ -61,6 +61,56 @@ void finish_plan(const mxa_decode_params_t *p, mxa_plan_t *plan) {
   plan->workspace_bytes = plan->needs_combine ? workspace_bytes(plan->units, plan->grid, p->D) : 0;
 }
 
+// Validate a run of `plan` and fill the launch description (len_add 0).
+mxa_status_t prepare_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+                            const int32_t *cache_seqlens, const mxa_decode_params_t *p, float scale, int causal,
+                            const mxa_plan_t *plan, void *workspace, size_t workspace_bytes, void *out,
+                            float *lse, DecodeLaunch *Lout) {
+  mxa_status_t st = check_shape(p);
+  if (st != MXA_OK) return st;
+  st = check_layout(p, block_table == nullptr);
+  if (st != MXA_OK) return st;
+  if (plan == nullptr) return MXA_ERR_INVALID_ARG;
+  if (p->B == 0) return MXA_OK;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || cache_seqlens == nullptr || out == nullptr)
+    return MXA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(cache_seqlens, 4) || (block_table && !aligned(block_table, 4)) || (lse && !aligned(lse, 4)))
+    return MXA_ERR_INVALID_ARG;
+  if (!isfinite(scale) || (causal != 0 && causal != 1)) return MXA_ERR_INVALID_ARG;
+
+  // Re-derive everything but the schedule choice from the shape.
+  mxa_plan_t use = *plan;
+  if (use.schedule != MXA_SCHED_UNIFORM && use.schedule != MXA_SCHED_BALANCED) return MXA_ERR_INVALID_ARG;
+  if (use.grid < 1 || use.num_splits < 1) return MXA_ERR_INVALID_ARG;
+  if (use.schedule == MXA_SCHED_BALANCED && (use.unit_cost < 0 || use.unit_cost > kMaxUnitCost))
+    return MXA_ERR_INVALID_ARG;
+  if (use.schedule == MXA_SCHED_UNIFORM) use.unit_cost = 0;
+  finish_plan(p, &use);
+  if (use.schedule == MXA_SCHED_UNIFORM && (long long)use.units * use.num_splits != use.grid)
+    return MXA_ERR_INVALID_ARG;
+  if (use.schedule == MXA_SCHED_BALANCED && p->B > kMaxBalancedRows) return MXA_ERR_UNSUPPORTED;
+  if (use.workspace_bytes > 0 && (workspace == nullptr || workspace_bytes < use.workspace_bytes ||
+                                  !aligned(workspace, 256)))
+    return MXA_ERR_WORKSPACE;
+
+  DecodeLaunch &L = *Lout;
+  L.q = q;
+  L.k_cache = k_cache;
+  L.v_cache = v_cache;
+  L.block_table = block_table;
+  L.seqlens = cache_seqlens;
+  L.out = out;
+  L.lse = lse;
+  L.workspace = workspace;
+  L.p = *p;
+  L.plan = use;
+  L.scale = scale;
+  L.causal = causal;
+  L.len_add = 0;
+  return MXA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -191,48 +241,37 @@ mxa_status_t mxa_decode_fwd_with_plan(const void *q, const void *k_cache, const 
                                       const mxa_decode_params_t *p, float scale, int causal,
                                       const mxa_plan_t *plan, void *workspace, size_t workspace_bytes,
                                       void *out, float *lse, void *stream) {
-  mxa_status_t st = check_shape(p);
-  if (st != MXA_OK) return st;
-  st = check_layout(p, block_table == nullptr);
-  if (st != MXA_OK) return st;
-  if (plan == nullptr) return MXA_ERR_INVALID_ARG;
-  if (p->B == 0) return MXA_OK;
-  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || cache_seqlens == nullptr || out == nullptr)
-    return MXA_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
-      !aligned(cache_seqlens, 4) || (block_table && !aligned(block_table, 4)) || (lse && !aligned(lse, 4)))
-    return MXA_ERR_INVALID_ARG;
-  if (!isfinite(scale) || (causal != 0 && causal != 1)) return MXA_ERR_INVALID_ARG;
-
-  // Re-derive everything but the schedule choice from the shape.
-  mxa_plan_t use = *plan;
-  if (use.schedule != MXA_SCHED_UNIFORM && use.schedule != MXA_SCHED_BALANCED) return MXA_ERR_INVALID_ARG;
-  if (use.grid < 1 || use.num_splits < 1) return MXA_ERR_INVALID_ARG;
-  if (use.schedule == MXA_SCHED_BALANCED && (use.unit_cost < 0 || use.unit_cost > kMaxUnitCost))
-    return MXA_ERR_INVALID_ARG;
-  if (use.schedule == MXA_SCHED_UNIFORM) use.unit_cost = 0;
-  finish_plan(p, &use);
-  if (use.schedule == MXA_SCHED_UNIFORM && (long long)use.units * use.num_splits != use.grid)
-    return MXA_ERR_INVALID_ARG;
-  if (use.schedule == MXA_SCHED_BALANCED && p->B > kMaxBalancedRows) return MXA_ERR_UNSUPPORTED;
-  if (use.workspace_bytes > 0 && (workspace == nullptr || workspace_bytes < use.workspace_bytes ||
-                                  !aligned(workspace, 256)))
-    return MXA_ERR_WORKSPACE;
-
   DecodeLaunch L;
-  L.q = q;
-  L.k_cache = k_cache;
-  L.v_cache = v_cache;
-  L.block_table = block_table;
-  L.seqlens = cache_seqlens;
-  L.out = out;
-  L.lse = lse;
-  L.workspace = workspace;
-  L.p = *p;
-  L.plan = use;
-  L.scale = scale;
-  L.causal = causal;
+  mxa_status_t st = prepare_decode(q, k_cache, v_cache, block_table, cache_seqlens, p, scale, causal, plan,
+                                   workspace, workspace_bytes, out, lse, &L);
+  if (st != MXA_OK || p->B == 0) return st;
   return launch_decode(L, static_cast<cudaStream_t>(stream));
+}
+
+mxa_status_t mxa_decode_fwd_append(const void *q, void *k_cache, void *v_cache, const void *k_new,
+                                   const void *v_new, const int32_t *block_table, const int32_t *cache_seqlens,
+                                   const mxa_decode_params_t *p, float scale, int causal, const mxa_plan_t *plan,
+                                   void *workspace, size_t workspace_bytes, void *out, float *lse,
+                                   void *stream) {
+  DecodeLaunch L;
+  mxa_status_t st = prepare_decode(q, k_cache, v_cache, block_table, cache_seqlens, p, scale, causal, plan,
+                                   workspace, workspace_bytes, out, lse, &L);
+  if (st != MXA_OK || p->B == 0) return st;
+  if (k_new == nullptr || v_new == nullptr) return MXA_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16)) return MXA_ERR_INVALID_ARG;
+  AppendLaunch A;
+  A.k_cache = k_cache;
+  A.v_cache = v_cache;
+  A.k_new = k_new;
+  A.v_new = v_new;
+  A.block_table = block_table;
+  A.seqlens = cache_seqlens;
+  A.p = *p;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_append(A, s);
+  if (st != MXA_OK) return st;
+  L.len_add = p->q_len;
+  return launch_decode(L, s);
 }
 
 mxa_status_t mxa_decode_fwd(const void *q, const void *k_cache, const void *v_cache,

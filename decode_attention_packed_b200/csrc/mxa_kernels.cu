@@ -85,7 +85,7 @@ __device__ __forceinline__ void cursor_enter_row(Cursor &c, const DecodeArgs &a,
   constexpr int T = block_tokens(D);
   c.L = L;
   c.nb = (L + T - 1) / T;
-  c.L_next = c.b + 1 < a.B ? a.seqlens[c.b + 1] : 0;  // consumed a segment later
+  c.L_next = c.b + 1 < a.B ? a.seqlens[c.b + 1] + a.len_add : 0;  // consumed a segment later
 }
 
 // The segment at the cursor (a contiguous block range of one unit); the
@@ -126,7 +126,7 @@ __device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
         cursor_enter_row<D>(c, a, clamp_len(c.L_next, a.max_seqlen_k));
         while (c.nb == 0 && c.b + 1 < a.B) {  // rows without keys hold no units
           ++c.b;
-          cursor_enter_row<D>(c, a, clamp_len(a.seqlens[c.b], a.max_seqlen_k));
+          cursor_enter_row<D>(c, a, clamp_len(a.seqlens[c.b] + a.len_add, a.max_seqlen_k));
         }
       } else {
         c.end = c.x;
@@ -160,7 +160,7 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
     const int u = blockIdx.x / a.splits, si = blockIdx.x % a.splits;
     c.b = u / HR;
     c.hr = u % HR;
-    c.L = clamp_len(a.seqlens[c.b], a.max_seqlen_k);
+    c.L = clamp_len(a.seqlens[c.b] + a.len_add, a.max_seqlen_k);
     c.nb = (c.L + T - 1) / T;
     const int beg = si * a.chunk_blocks, end = min(beg + a.chunk_blocks, c.nb);
     c.blk = beg;
@@ -175,7 +175,7 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
   const int lo = min(lane * chunk, a.B), hi = min(lo + chunk, a.B);
   int sum = 0;
   for (int i = lo; i < hi; ++i) {
-    const int L = clamp_len(a.seqlens[i], a.max_seqlen_k);
+    const int L = clamp_len(a.seqlens[i] + a.len_add, a.max_seqlen_k);
     lens[i] = L;
     const int nb = (L + T - 1) / T;
     const int w = nb > 0 ? nb + V : 0;  // positions of one unit of row i
@@ -973,10 +973,10 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
   // their empty result.
   if (a.schedule == MXA_SCHED_BALANCED) {
     for (int u = blockIdx.x; u < a.units; u += gridDim.x)
-      if (clamp_len(a.seqlens[u / HR], a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, lane);
+      if (clamp_len(a.seqlens[u / HR] + a.len_add, a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, lane);
   } else if (blockIdx.x % a.splits == 0) {
     const int u = blockIdx.x / a.splits;
-    if (clamp_len(a.seqlens[u / HR], a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, lane);
+    if (clamp_len(a.seqlens[u / HR] + a.len_add, a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, lane);
   }
 
   // Tag the arrival counters of this CTA's split units with this launch's
@@ -1236,6 +1236,45 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // ---------------------------------------------------------------------------
+// Append: row b's new token t (k_new / v_new [B, q_len, Hkv, D]) goes to
+// logical position cache_seqlens[b] + t of the row, before the attention
+// kernel that follows on the stream reads the cache.  One warp per
+// (b, t, KV head); its lanes copy the K and V rows 16 bytes each.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128)
+    mxa_append_kernel(uint16_t *__restrict__ k_cache, uint16_t *__restrict__ v_cache,
+                      const uint16_t *__restrict__ k_new, const uint16_t *__restrict__ v_new,
+                      const int32_t *__restrict__ block_table, const int32_t *__restrict__ seqlens, int B,
+                      int q_len, int Hkv, int page_size, int mpps, int contiguous, int max_seqlen_k) {
+  constexpr int CH = D * 2 / 16;  // 16-byte chunks of one head's row
+  // The new tokens and the lengths may come from the kernel this launch
+  // depends on; the attention kernel after this one may start its prologue.
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const long long rows = (long long)B * q_len * Hkv;
+  const long long r = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows || lane >= 2 * CH) return;
+  const int h = (int)(r % Hkv), t = (int)((r / Hkv) % q_len), b = (int)(r / ((long long)Hkv * q_len));
+  const int pos = seqlens[b] + t;
+  if (pos < 0 || pos >= max_seqlen_k) return;  // no room: not written
+  long long token;  // the token's row in the pool
+  if (contiguous) {
+    if (pos >= page_size) return;
+    token = (long long)b * page_size + pos;
+  } else {
+    const int lp = pos / page_size;
+    if (lp >= mpps) return;
+    token = (long long)block_table[(size_t)b * mpps + lp] * page_size + pos % page_size;
+  }
+  const bool is_v = lane >= CH;
+  const int c = is_v ? lane - CH : lane;
+  const uint4 v = reinterpret_cast<const uint4 *>(is_v ? v_new : k_new)[(size_t)r * CH + c];
+  reinterpret_cast<uint4 *>(is_v ? v_cache : k_cache)[((size_t)token * Hkv + h) * CH + c] = v;
+}
+
+// ---------------------------------------------------------------------------
 // mxa_combine: split results in the uniform layout o_part[S, B, q_len, Hq, D],
 // lse_part[S, B, Hq, q_len].  One warp per (b, t, h) row.
 // ---------------------------------------------------------------------------
@@ -1380,6 +1419,7 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
   if (a.chunk_blocks < 1) a.chunk_blocks = 1;
   a.units = plan.units;
   a.unit_cost = plan.schedule == MXA_SCHED_BALANCED ? plan.unit_cost : 0;
+  a.len_add = L.len_add;
   a.epoch = next_epoch();
   if (plan.workspace_bytes > 0) {
     uint8_t *ws = static_cast<uint8_t *>(L.workspace);
@@ -1415,6 +1455,35 @@ mxa_status_t launch_decode(const DecodeLaunch &L, cudaStream_t stream) {
   if (L.p.D == 128) return bf16 ? launch_typed<128, true>(L, stream) : launch_typed<128, false>(L, stream);
   if (L.p.D == 64) return bf16 ? launch_typed<64, true>(L, stream) : launch_typed<64, false>(L, stream);
   return MXA_ERR_UNSUPPORTED;
+}
+
+mxa_status_t launch_append(const AppendLaunch &L, cudaStream_t stream) {
+  const mxa_decode_params_t &p = L.p;
+  const long long rows = (long long)p.B * p.q_len * p.Hkv;
+  if (rows == 0) return MXA_OK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((rows + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int contiguous = L.block_table == nullptr ? 1 : 0;
+  uint16_t *kc = static_cast<uint16_t *>(L.k_cache), *vc = static_cast<uint16_t *>(L.v_cache);
+  const uint16_t *kn = static_cast<const uint16_t *>(L.k_new), *vn = static_cast<const uint16_t *>(L.v_new);
+  cudaError_t e;
+  if (p.D == 128)
+    e = cudaLaunchKernelEx(&cfg, mxa_append_kernel<128>, kc, vc, kn, vn, L.block_table, L.seqlens, p.B, p.q_len,
+                           p.Hkv, p.page_size, p.max_pages_per_seq, contiguous, p.max_seqlen_k);
+  else if (p.D == 64)
+    e = cudaLaunchKernelEx(&cfg, mxa_append_kernel<64>, kc, vc, kn, vn, L.block_table, L.seqlens, p.B, p.q_len,
+                           p.Hkv, p.page_size, p.max_pages_per_seq, contiguous, p.max_seqlen_k);
+  else
+    return MXA_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return MXA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? MXA_OK : MXA_ERR_CUDA;
 }
 
 mxa_status_t launch_combine(const float *o_part, const float *lse_part, int num_splits, int B,

@@ -39,6 +39,7 @@ struct DecodeArgs {
   int chunk_blocks;            // UNIFORM: blocks per split
   int units;
   int unit_cost;               // BALANCED: fixed cost of a unit, in KV blocks
+  int len_add;                 // keys each row holds beyond cache_seqlens (appended this call)
   unsigned int epoch;          // tags this launch's arrival counts
 };
 
@@ -53,7 +54,20 @@ struct DecodeLaunch {
   mxa_plan_t plan;
   float scale;
   int causal;
+  int len_add;  // q_len when the call appends the new tokens first, else 0
 };
+
+// Everything launch_append needs: write k_new / v_new [B, q_len, Hkv, D] at
+// logical positions cache_seqlens[b] + t of each row.
+struct AppendLaunch {
+  void *k_cache, *v_cache;
+  const void *k_new, *v_new;
+  const int32_t *block_table, *seqlens;
+  mxa_decode_params_t p;
+};
+
+// Launch the append kernel (before a decode that reads the appended keys).
+mxa_status_t launch_append(const AppendLaunch &L, cudaStream_t stream);
 
 // Launch the split kernel (split units are merged inside it).
 mxa_status_t launch_decode(const DecodeLaunch &L, cudaStream_t stream);

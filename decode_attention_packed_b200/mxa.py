@@ -30,7 +30,7 @@ MXA_SCHED_UNIFORM, MXA_SCHED_BALANCED = 0, 1
 EXPORTED = ("mxa_status_string", "mxa_should_pack_gqa", "mxa_num_splits_heuristic", "mxa_plan",
             "mxa_plan_balanced",
             "mxa_decode_fwd", "mxa_decode_fwd_with_plan", "mxa_combine", "mxa_device_error",
-            "mxa_decode_fwd_noalloc")
+            "mxa_decode_fwd_noalloc", "mxa_decode_fwd_append")
 
 
 class mxa_decode_params_t(ctypes.Structure):
@@ -70,6 +70,10 @@ _lib.mxa_decode_fwd_with_plan.argtypes = [_P, _P, _P, _P, _P, ctypes.POINTER(mxa
                                           ctypes.c_float, _I, ctypes.POINTER(mxa_plan_t), _P,
                                           ctypes.c_size_t, _P, _P, _P]
 _lib.mxa_decode_fwd_with_plan.restype = _I
+_lib.mxa_decode_fwd_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(mxa_decode_params_t),
+                                       ctypes.c_float, _I, ctypes.POINTER(mxa_plan_t), _P, ctypes.c_size_t,
+                                       _P, _P, _P]
+_lib.mxa_decode_fwd_append.restype = _I
 _lib.mxa_decode_fwd_noalloc.argtypes = [_P, _P, _P, _P, _P, ctypes.POINTER(mxa_decode_params_t),
                                         ctypes.c_float, _I, _I, _P, _P, _P]
 _lib.mxa_decode_fwd_noalloc.restype = _I
@@ -150,6 +154,17 @@ def mxa_decode_fwd_with_plan(q, k_cache, v_cache, block_table, cache_seqlens, pa
            "mxa_decode_fwd_with_plan")
 
 
+def mxa_decode_fwd_append(q, k_cache, v_cache, k_new, v_new, block_table, cache_seqlens, params, scale,
+                          causal, plan, workspace, out, lse, stream=None) -> None:
+    """Write k_new / v_new [B, q_len, Hkv, D] at positions cache_seqlens[b] + t of
+    the cache, then decode over cache_seqlens[b] + q_len keys (see mxa.h)."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.mxa_decode_fwd_append(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new),
+                                      _ptr(block_table), _ptr(cache_seqlens), ctypes.byref(params),
+                                      float(scale), int(causal), ctypes.byref(plan), _ptr(workspace), ws_bytes,
+                                      _ptr(out), _ptr(lse), _stream(stream)), "mxa_decode_fwd_append")
+
+
 def mxa_decode_fwd_noalloc(q, k_cache, v_cache, block_table, cache_seqlens, params, scale, causal,
                            num_splits, out, lse, stream=None) -> None:
     """Decode with the library's fixed 16 MiB scratch array instead of a
@@ -223,8 +238,12 @@ def prepare(q, k_cache, block_table, *, max_seqlen_k=None, num_splits=0, plan=No
 
 def decode(q, k_cache, v_cache, block_table, cache_seqlens, *, scale=None, causal=False,
            num_splits=0, max_seqlen_k=None, out=None, lse=None, prepared: Optional[Prepared] = None,
-           return_lse=True, stream=None):
-    """out [B, q_len, Hq, D] (and lse [B, Hq, q_len] fp32) for one decode step."""
+           return_lse=True, stream=None, k_new=None, v_new=None):
+    """out [B, q_len, Hq, D] (and lse [B, Hq, q_len] fp32) for one decode step.
+
+    With k_new / v_new [B, q_len, Hkv, D] the step first writes them into the
+    cache at positions cache_seqlens[b] + t and attends to cache_seqlens[b] +
+    q_len keys; max_seqlen_k must then bound those lengths."""
     if scale is None:
         scale = q.shape[-1] ** -0.5
     if prepared is None:
@@ -234,6 +253,12 @@ def decode(q, k_cache, v_cache, block_table, cache_seqlens, *, scale=None, causa
     if lse is None and return_lse:
         B, q_len, Hq, _ = q.shape
         lse = torch.empty((B, Hq, q_len), dtype=torch.float32, device=q.device)
-    mxa_decode_fwd_with_plan(q, k_cache, v_cache, block_table, cache_seqlens, prepared.params, scale,
-                             causal, prepared.plan, prepared.workspace, out, lse, stream)
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
+    if k_new is None:
+        mxa_decode_fwd_with_plan(q, k_cache, v_cache, block_table, cache_seqlens, prepared.params, scale,
+                                 causal, prepared.plan, prepared.workspace, out, lse, stream)
+    else:
+        mxa_decode_fwd_append(q, k_cache, v_cache, k_new, v_new, block_table, cache_seqlens, prepared.params,
+                              scale, causal, prepared.plan, prepared.workspace, out, lse, stream)
     return out, lse

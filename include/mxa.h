@@ -206,6 +206,30 @@ MXA_API mxa_status_t mxa_decode_fwd_with_plan(const void *q, const void *k_cache
                                       size_t workspace_bytes, void *out, float *lse,
                                       void *stream);
 
+/* Append the new tokens' keys and values to the cache, then decode, in one
+ * call: the k / v arguments of flash_attn_with_kvcache next to cache_seqlens
+ * ("Flash-Attention GQA 性能调优: pack_gqa 与 num_splits", its usage example)
+ * and the paged KV append of "MXFlashAttn 1.4.0" (能力矩阵).
+ *   k_new, v_new : device [B, q_len, Hkv, D] dtype, read only: the q_len new
+ *                  tokens of each row (the tokens the queries belong to)
+ *   cache_seqlens: device [B], read only: L_b, the keys the cache holds before
+ *                  this call (not updated; the caller adds q_len afterwards)
+ *   k_cache, v_cache: written: row b's new token t goes to logical position
+ *                  L_b + t (page block_table[b][(L_b + t) / page_size], slot
+ *                  (L_b + t) % page_size; contiguous: row b, slot L_b + t)
+ * Every query row then attends to the first L_b + q_len keys; with causal = 1
+ * query t sees the first L_b + t + 1.  params->max_seqlen_k bounds L_b + q_len
+ * (tokens that would land at or past it, or past the row's block-table
+ * width, are not written).  The plan is that of mxa_plan for `params`.  Two
+ * kernels run on `stream`: the append, then the attention, which starts its
+ * prologue early and reads the cache only once the append has completed.
+ * Other arguments and errors as mxa_decode_fwd_with_plan. */
+MXA_API mxa_status_t mxa_decode_fwd_append(const void *q, void *k_cache, void *v_cache, const void *k_new,
+                                           const void *v_new, const int32_t *block_table,
+                                           const int32_t *cache_seqlens, const mxa_decode_params_t *params,
+                                           float scale, int causal, const mxa_plan_t *plan, void *workspace,
+                                           size_t workspace_bytes, void *out, float *lse, void *stream);
+
 /* Decode without any device allocation, for callers that cannot allocate.
  * (An addition of this library; the source pages have no counterpart.)
  *
