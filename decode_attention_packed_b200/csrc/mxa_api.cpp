@@ -108,6 +108,7 @@ mxa_status_t prepare_decode(const void *q, const void *k_cache, const void *v_ca
   L.scale = scale;
   L.causal = causal;
   L.len_add = 0;
+  L.k_new = L.v_new = nullptr;
   return MXA_OK;
 }
 
@@ -259,19 +260,10 @@ mxa_status_t mxa_decode_fwd_append(const void *q, void *k_cache, void *v_cache, 
   if (st != MXA_OK || p->B == 0) return st;
   if (k_new == nullptr || v_new == nullptr) return MXA_ERR_INVALID_ARG;
   if (!aligned(k_new, 16) || !aligned(v_new, 16)) return MXA_ERR_INVALID_ARG;
-  AppendLaunch A;
-  A.k_cache = k_cache;
-  A.v_cache = v_cache;
-  A.k_new = k_new;
-  A.v_new = v_new;
-  A.block_table = block_table;
-  A.seqlens = cache_seqlens;
-  A.p = *p;
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_append(A, s);
-  if (st != MXA_OK) return st;
   L.len_add = p->q_len;
-  return launch_decode(L, s);
+  L.k_new = k_new;
+  L.v_new = v_new;
+  return launch_decode(L, static_cast<cudaStream_t>(stream));
 }
 
 mxa_status_t mxa_decode_fwd(const void *q, const void *k_cache, const void *v_cache,

@@ -267,7 +267,9 @@ __device__ __forceinline__ int bt_entry(const DecodeArgs &a, int b, int p, int n
   return p < npages ? a.block_table[(size_t)b * a.mpps + p] : 0;
 }
 
-template <int D, bool kBf16>
+// kAppend: the call appends new tokens to the cache (len_add > 0); the plain
+// decode instance carries none of that code.
+template <int D, bool kBf16, bool kAppend>
 __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *smem, int lane) {
   constexpr int T = block_tokens(D);
   constexpr int CH = D / 64;
@@ -345,12 +347,39 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
     w.wb = bt_entry(a, s.b, w.base + 32 + lane, a.mpps);
   };
 
+  // Copy the appended tokens at positions [p0, p1) of segment `s`'s row into
+  // the caches for its KV head: 16 bytes per lane, K and V rows side by side.
+  // Every lane takes part in the page lookups (shuffles).
+  auto write_new_tokens = [&](const SegmentDesc &s, const Window &w, int n0, int p0, int p1) {
+    constexpr int CW = D * 2 / 16;  // 16-byte chunks of one head's row
+    for (int p = p0; p < p1; ++p) {
+      long long token;
+      if (a.contiguous) {
+        token = (long long)s.b * ps + p;
+      } else {
+        const int idx = p / ps - w.base;
+        const int va = __shfl_sync(0xffffffffu, w.wa, idx & 31);
+        const int vb = __shfl_sync(0xffffffffu, w.wb, idx & 31);
+        token = (long long)(idx < 32 ? va : vb) * ps + p % ps;
+      }
+      if (lane < 2 * CW) {
+        const bool is_v = lane >= CW;
+        const int c = is_v ? lane - CW : lane;
+        const size_t src = ((size_t)(s.b * a.q_len + (p - n0)) * a.Hkv + s.h) * CW + c;
+        const uint4 v = reinterpret_cast<const uint4 *>(is_v ? a.v_new : a.k_new)[src];
+        reinterpret_cast<uint4 *>(is_v ? a.v_cache_w : a.k_cache_w)[((size_t)token * a.Hkv + s.h) * CW + c] = v;
+      }
+    }
+  };
+
   int it = 0;     // KV stages issued
   int seg_k = 0;  // segments published
   bool ok = true;
   if (more()) {
     SegmentDesc seg = take();
     seg.last = more() ? 0 : 1;
+    int new0 = 0;  // first appended position of the row
+    if constexpr (kAppend) new0 = a.seqlens[seg.b];
     Window win;
     load_window(seg, win);
     if (!warp_wait_bounded(qempty, 1, &g_mxa_err, kErrWaitQ, lane)) ok = false;  // first use: free
@@ -362,6 +391,7 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
       bool have_next = false, next_known = false, q_next = false;
       SegmentDesc nseg;
       Window nwin;
+      int nnew0 = 0;
       for (int blk = seg.blk_beg; blk < seg.blk_end; ++blk) {
         const int s = it % kStages;
         const int k = it / kStages;
@@ -378,6 +408,17 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
                                lane)) {
           ok = false;
           break;
+        }
+        // Tokens this call appends that fall in this block go into the cache
+        // first (this unit's KV head), and are fenced against the loads below.
+        if constexpr (kAppend) {
+          const int n0 = new0 < 0 ? 0 : new0, n1 = min(new0 + a.len_add, seg.L);
+          const int p0 = max(n0, tok0), p1 = min(n1, tok0 + T);
+          if (p1 > p0) {
+            write_new_tokens(seg, win, new0, p0, p1);
+            fence_proxy_async_global();
+            __syncwarp();
+          }
         }
         if (lane == 0) mbar_arrive_expect_tx(bar_addr(smem, D, B_FULL(s)), (uint32_t)nbox * bt * D * 2 * 2);
         __syncwarp();
@@ -412,6 +453,7 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
           if (have_next) {
             nseg = take();
             nseg.last = more() ? 0 : 1;
+            if constexpr (kAppend) nnew0 = a.seqlens[nseg.b];
             load_window(nseg, nwin);
           }
         }
@@ -437,6 +479,7 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
       }
       seg = nseg;
       win = nwin;
+      new0 = nnew0;
     }
   }
 
@@ -1196,7 +1239,7 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
 // ---------------------------------------------------------------------------
 // The split kernel
 // ---------------------------------------------------------------------------
-template <int D, bool kBf16>
+template <int D, bool kBf16, bool kAppend>
 __global__ void __launch_bounds__(kThreads, 2)
     mxa_split_kernel(const __grid_constant__ TmapPair tm, const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -1227,51 +1270,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   // warps).  The math warps touch shared memory only.
   grid_launch_dependents();
   if (warp == kProducerWarp) {
-    producer_warp<D, kBf16>(tm, a, smem, lane);
+    producer_warp<D, kBf16, kAppend>(tm, a, smem, lane);
   } else if (warp == kEpilogueWarp) {
     epilogue_warp<D, kBf16>(a, smem, lane);
   } else {
     math_warps<D, kBf16>(a, smem, warp, lane);
   }
-}
-
-// ---------------------------------------------------------------------------
-// Append: row b's new token t (k_new / v_new [B, q_len, Hkv, D]) goes to
-// logical position cache_seqlens[b] + t of the row, before the attention
-// kernel that follows on the stream reads the cache.  One warp per
-// (b, t, KV head); its lanes copy the K and V rows 16 bytes each.
-// ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(128)
-    mxa_append_kernel(uint16_t *__restrict__ k_cache, uint16_t *__restrict__ v_cache,
-                      const uint16_t *__restrict__ k_new, const uint16_t *__restrict__ v_new,
-                      const int32_t *__restrict__ block_table, const int32_t *__restrict__ seqlens, int B,
-                      int q_len, int Hkv, int page_size, int mpps, int contiguous, int max_seqlen_k) {
-  constexpr int CH = D * 2 / 16;  // 16-byte chunks of one head's row
-  // The new tokens and the lengths may come from the kernel this launch
-  // depends on; the attention kernel after this one may start its prologue.
-  grid_dependency_wait();
-  grid_launch_dependents();
-  const long long rows = (long long)B * q_len * Hkv;
-  const long long r = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (r >= rows || lane >= 2 * CH) return;
-  const int h = (int)(r % Hkv), t = (int)((r / Hkv) % q_len), b = (int)(r / ((long long)Hkv * q_len));
-  const int pos = seqlens[b] + t;
-  if (pos < 0 || pos >= max_seqlen_k) return;  // no room: not written
-  long long token;  // the token's row in the pool
-  if (contiguous) {
-    if (pos >= page_size) return;
-    token = (long long)b * page_size + pos;
-  } else {
-    const int lp = pos / page_size;
-    if (lp >= mpps) return;
-    token = (long long)block_table[(size_t)b * mpps + lp] * page_size + pos % page_size;
-  }
-  const bool is_v = lane >= CH;
-  const int c = is_v ? lane - CH : lane;
-  const uint4 v = reinterpret_cast<const uint4 *>(is_v ? v_new : k_new)[(size_t)r * CH + c];
-  reinterpret_cast<uint4 *>(is_v ? v_cache : k_cache)[((size_t)token * Hkv + h) * CH + c] = v;
 }
 
 // ---------------------------------------------------------------------------
@@ -1363,13 +1367,13 @@ bool encode_kv_map(CUtensorMap *m, const void *base, int D, int Hkv, long long p
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool kBf16>
+template <int D, bool kBf16, bool kAppend>
 cudaError_t prepare_split_kernel(int device) {
   static std::mutex mu;
   static bool done[kMaxDevices] = {};
   std::lock_guard<std::mutex> lock(mu);
   if (device >= 0 && device < kMaxDevices && done[device]) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(mxa_split_kernel<D, kBf16>,
+  cudaError_t e = cudaFuncSetAttribute(mxa_split_kernel<D, kBf16, kAppend>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_total(D));
   if (e == cudaSuccess && device >= 0 && device < kMaxDevices) done[device] = true;
   return e;
@@ -1390,7 +1394,10 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
   const mxa_plan_t &plan = L.plan;
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return MXA_ERR_CUDA;
-  if (prepare_split_kernel<D, kBf16>(device) != cudaSuccess) return MXA_ERR_CUDA;
+  const bool append = L.len_add > 0;
+  if ((append ? prepare_split_kernel<D, kBf16, true>(device) : prepare_split_kernel<D, kBf16, false>(device)) !=
+      cudaSuccess)
+    return MXA_ERR_CUDA;
 
   DecodeArgs a{};
   a.q = L.q;
@@ -1420,6 +1427,10 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
   a.units = plan.units;
   a.unit_cost = plan.schedule == MXA_SCHED_BALANCED ? plan.unit_cost : 0;
   a.len_add = L.len_add;
+  a.k_new = static_cast<const uint16_t *>(L.k_new);
+  a.v_new = static_cast<const uint16_t *>(L.v_new);
+  a.k_cache_w = static_cast<uint16_t *>(const_cast<void *>(L.k_cache));
+  a.v_cache_w = static_cast<uint16_t *>(const_cast<void *>(L.v_cache));
   a.epoch = next_epoch();
   if (plan.workspace_bytes > 0) {
     uint8_t *ws = static_cast<uint8_t *>(L.workspace);
@@ -1444,7 +1455,9 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, mxa_split_kernel<D, kBf16>, tm, a) != cudaSuccess) return MXA_ERR_CUDA;
+  const cudaError_t e = append ? cudaLaunchKernelEx(&cfg, mxa_split_kernel<D, kBf16, true>, tm, a)
+                               : cudaLaunchKernelEx(&cfg, mxa_split_kernel<D, kBf16, false>, tm, a);
+  if (e != cudaSuccess) return MXA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? MXA_OK : MXA_ERR_CUDA;
 }
 
@@ -1455,35 +1468,6 @@ mxa_status_t launch_decode(const DecodeLaunch &L, cudaStream_t stream) {
   if (L.p.D == 128) return bf16 ? launch_typed<128, true>(L, stream) : launch_typed<128, false>(L, stream);
   if (L.p.D == 64) return bf16 ? launch_typed<64, true>(L, stream) : launch_typed<64, false>(L, stream);
   return MXA_ERR_UNSUPPORTED;
-}
-
-mxa_status_t launch_append(const AppendLaunch &L, cudaStream_t stream) {
-  const mxa_decode_params_t &p = L.p;
-  const long long rows = (long long)p.B * p.q_len * p.Hkv;
-  if (rows == 0) return MXA_OK;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((rows + 3) / 4));
-  cfg.blockDim = dim3(128);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const int contiguous = L.block_table == nullptr ? 1 : 0;
-  uint16_t *kc = static_cast<uint16_t *>(L.k_cache), *vc = static_cast<uint16_t *>(L.v_cache);
-  const uint16_t *kn = static_cast<const uint16_t *>(L.k_new), *vn = static_cast<const uint16_t *>(L.v_new);
-  cudaError_t e;
-  if (p.D == 128)
-    e = cudaLaunchKernelEx(&cfg, mxa_append_kernel<128>, kc, vc, kn, vn, L.block_table, L.seqlens, p.B, p.q_len,
-                           p.Hkv, p.page_size, p.max_pages_per_seq, contiguous, p.max_seqlen_k);
-  else if (p.D == 64)
-    e = cudaLaunchKernelEx(&cfg, mxa_append_kernel<64>, kc, vc, kn, vn, L.block_table, L.seqlens, p.B, p.q_len,
-                           p.Hkv, p.page_size, p.max_pages_per_seq, contiguous, p.max_seqlen_k);
-  else
-    return MXA_ERR_UNSUPPORTED;
-  if (e != cudaSuccess) return MXA_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? MXA_OK : MXA_ERR_CUDA;
 }
 
 mxa_status_t launch_combine(const float *o_part, const float *lse_part, int num_splits, int B,

@@ -39,7 +39,11 @@ struct DecodeArgs {
   int chunk_blocks;            // UNIFORM: blocks per split
   int units;
   int unit_cost;               // BALANCED: fixed cost of a unit, in KV blocks
-  int len_add;                 // keys each row holds beyond cache_seqlens (appended this call)
+  int len_add;                 // new tokens appended to each row this call (0: none)
+  const uint16_t *k_new;       // [B, q_len, Hkv, D]: the appended tokens' keys (len_add > 0)
+  const uint16_t *v_new;       //   and values
+  uint16_t *k_cache_w;         // the caches, written at the appended positions
+  uint16_t *v_cache_w;
   unsigned int epoch;          // tags this launch's arrival counts
 };
 
@@ -55,19 +59,8 @@ struct DecodeLaunch {
   float scale;
   int causal;
   int len_add;  // q_len when the call appends the new tokens first, else 0
+  const void *k_new, *v_new;  // [B, q_len, Hkv, D] when len_add > 0
 };
-
-// Everything launch_append needs: write k_new / v_new [B, q_len, Hkv, D] at
-// logical positions cache_seqlens[b] + t of each row.
-struct AppendLaunch {
-  void *k_cache, *v_cache;
-  const void *k_new, *v_new;
-  const int32_t *block_table, *seqlens;
-  mxa_decode_params_t p;
-};
-
-// Launch the append kernel (before a decode that reads the appended keys).
-mxa_status_t launch_append(const AppendLaunch &L, cudaStream_t stream);
 
 // Launch the split kernel (split units are merged inside it).
 mxa_status_t launch_decode(const DecodeLaunch &L, cudaStream_t stream);

@@ -220,9 +220,10 @@ MXA_API mxa_status_t mxa_decode_fwd_with_plan(const void *q, const void *k_cache
  * Every query row then attends to the first L_b + q_len keys; with causal = 1
  * query t sees the first L_b + t + 1.  params->max_seqlen_k bounds L_b + q_len
  * (tokens that would land at or past it, or past the row's block-table
- * width, are not written).  The plan is that of mxa_plan for `params`.  Two
- * kernels run on `stream`: the append, then the attention, which starts its
- * prologue early and reads the cache only once the append has completed.
+ * width, are not written).  The plan is that of mxa_plan for `params`.  One
+ * kernel runs on `stream`: the CTA that streams the block holding an
+ * appended token writes the token into the cache (for its KV head) and then
+ * loads the block, so each token is written before it is read.
  * Other arguments and errors as mxa_decode_fwd_with_plan. */
 MXA_API mxa_status_t mxa_decode_fwd_append(const void *q, void *k_cache, void *v_cache, const void *k_new,
                                            const void *v_new, const int32_t *block_table,
