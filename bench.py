@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--num-splits", type=int, default=None)
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--append", action="store_true",
+                    help="each step also appends the step's q_len new tokens per row to the cache "
+                         "(mxa_decode_fwd_append) before attending")
     return ap.parse_args()
 
 
@@ -265,12 +268,25 @@ def main():
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=dev)
     nbytes = algorithmic_bytes(inp)
+    if args.append:  # the new tokens are read and written once more
+        nbytes["total"] += 2 * 2 * w.B * w.q_len * w.Hkv * w.D * inp.q.element_size()
     launches_per_call = 1  # the split kernel merges split units itself
+
+    if args.append:
+        # the rows' last q_len keys arrive as this step's new tokens: the call
+        # writes them (the same values each step) and attends to all keys
+        sl_before = (sl - w.q_len).clamp(min=0)
+        k_new = torch.randn((w.B, w.q_len, w.Hkv, w.D), device=dev).to(q.dtype)
+        v_new = torch.randn_like(k_new)
 
     def call(i):
         k, v = pools[i % N_POOLS]
-        mxa.mxa_decode_fwd_with_plan(q, k, v, bt, sl, prep.params, w.scale, w.causal, prep.plan,
-                                     prep.workspace, out, lse, stream)
+        if args.append:
+            mxa.mxa_decode_fwd_append(q, k, v, k_new, v_new, bt, sl_before, prep.params, w.scale, w.causal,
+                                      prep.plan, prep.workspace, out, lse, stream)
+        else:
+            mxa.mxa_decode_fwd_with_plan(q, k, v, bt, sl, prep.params, w.scale, w.causal, prep.plan,
+                                         prep.workspace, out, lse, stream)
 
     def barrier():
         if world > 1:
@@ -311,7 +327,7 @@ def main():
     # buffered, and events order each buffer's copy-in, decode and copy-out.
     hq = inp.q.pin_memory()
     hbt = None if inp.block_table is None else inp.block_table.pin_memory()
-    hsl = inp.cache_seqlens.pin_memory()
+    hsl = ((inp.cache_seqlens - w.q_len).clamp(min=0) if args.append else inp.cache_seqlens).pin_memory()
     h2d = hq.numel() * hq.element_size() + hsl.numel() * 4 + (0 if hbt is None else hbt.numel() * 4)
     d2h = out.numel() * out.element_size() + lse.numel() * 4
     e2e_steps = max(1, min(args.steps, 2000))
@@ -340,8 +356,12 @@ def main():
         stream.wait_event(sd["copied"])
         stream.wait_event(sd["read"])  # the read-back two steps back is done with these outputs
         k, v = pools[i % N_POOLS]
-        mxa.mxa_decode_fwd_with_plan(sd["q"], k, v, sd["bt"], sd["sl"], prep.params, w.scale, w.causal,
-                                     prep.plan, prep.workspace, sd["out"], sd["lse"], stream)
+        if args.append:
+            mxa.mxa_decode_fwd_append(sd["q"], k, v, k_new, v_new, sd["bt"], sd["sl"], prep.params, w.scale,
+                                      w.causal, prep.plan, prep.workspace, sd["out"], sd["lse"], stream)
+        else:
+            mxa.mxa_decode_fwd_with_plan(sd["q"], k, v, sd["bt"], sd["sl"], prep.params, w.scale, w.causal,
+                                         prep.plan, prep.workspace, sd["out"], sd["lse"], stream)
         sd["decoded"].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(sd["decoded"])
@@ -390,11 +410,12 @@ def main():
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic",
-        "config": workload_config(w, nbytes, world),
+        "config": dict(workload_config(w, nbytes, world), append=bool(args.append)),
         "plan": prep.plan.as_dict(),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": MEASURED_TRAFFIC.get(kernel_source_hash()) if w.name == DEFAULT_WORKLOAD else None,
+                     "traffic": MEASURED_TRAFFIC.get(kernel_source_hash())
+                     if w.name == DEFAULT_WORKLOAD and not args.append else None,
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                      else "fallback 6.65 TB/s",
                      "kernel": "mxa_split_kernel (one launch per call; split units merged inside)"},
