@@ -39,7 +39,7 @@ METRIC = "decode-attn µs/call and KV-read GB/s as % of B200 HBM peak (1 GPU)"
 # workload, from an ncu capture (profiles/mxa_split_kernel_gqa_decode.md),
 # keyed by a hash of the kernel sources it was taken on: once the kernel
 # changes the number no longer applies and the bench reports null.
-MEASURED_TRAFFIC = {"750bd1dbedb7eb1e": 249119488}
+MEASURED_TRAFFIC = {"86f2af96b916765d": 248780544}
 DEFAULT_WORKLOAD = "gqa_decode"
 FALLBACK_HBM_GBS = 6650.0
 N_POOLS = 3
