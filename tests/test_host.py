@@ -202,6 +202,27 @@ def test_run_refuses_bad_arguments_before_launch():
     assert _run_with_plan(p0, mxa.mxa_plan(p0, 1, sm_count=148)) == MXA_OK
 
 
+def test_append_refuses_bad_arguments_before_launch():
+    # the append entry point checks like the plain run, and needs both new-token arrays
+    p = params()
+    plan = mxa.mxa_plan(p, 0, sm_count=148)
+    f = lambda x: None if x is None else ctypes.c_void_p(x * 4096)
+    call = lambda **kw: mxa._lib.mxa_decode_fwd_append(
+        f(kw.get("q", 1)), f(1), f(1), f(kw.get("k_new", 1)), f(kw.get("v_new", 1)), f(1), f(1),
+        ctypes.byref(p), 0.125, 0, ctypes.byref(plan), f(1), 1 << 30, f(1), None, None)
+    assert call(k_new=None) == MXA_ERR_INVALID_ARG
+    assert call(v_new=None) == MXA_ERR_INVALID_ARG
+    assert call(q=None) == MXA_ERR_INVALID_ARG
+    misaligned = mxa._lib.mxa_decode_fwd_append(f(1), f(1), f(1), ctypes.c_void_p(4096 + 8), f(1), f(1), f(1),
+                                                ctypes.byref(p), 0.125, 0, ctypes.byref(plan), f(1), 1 << 30,
+                                                f(1), None, None)
+    assert misaligned == MXA_ERR_INVALID_ARG
+    p0 = params(B=0)
+    assert mxa._lib.mxa_decode_fwd_append(None, None, None, None, None, None, None, ctypes.byref(p0), 0.125, 0,
+                                          ctypes.byref(mxa.mxa_plan(p0, 1, sm_count=148)), None, 0, None, None,
+                                          None) == MXA_OK
+
+
 def test_combine_refuses_bad_arguments():
     f = lambda x: None if x is None else ctypes.c_void_p(x * 4096)
     c = mxa._lib.mxa_combine
