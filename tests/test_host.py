@@ -218,9 +218,9 @@ def test_append_refuses_bad_arguments_before_launch():
                                                 f(1), None, None)
     assert misaligned == MXA_ERR_INVALID_ARG
     p0 = params(B=0)
-    assert mxa._lib.mxa_decode_fwd_append(None, None, None, None, None, None, None, ctypes.byref(p0), 0.125, 0,
+    assert mxa._lib.mxa_decode_fwd_append(None, None, None, None, None, f(1), None, ctypes.byref(p0), 0.125, 0,
                                           ctypes.byref(mxa.mxa_plan(p0, 1, sm_count=148)), None, 0, None, None,
-                                          None) == MXA_OK
+                                          None) == MXA_OK  # nothing to do for B = 0 (paged layout)
 
 
 def test_combine_refuses_bad_arguments():
