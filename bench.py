@@ -39,7 +39,7 @@ METRIC = "decode-attn µs/call and KV-read GB/s as % of B200 HBM peak (1 GPU)"
 # workload, from an ncu capture (profiles/mxa_split_kernel_gqa_decode.md),
 # keyed by a hash of the kernel sources it was taken on: once the kernel
 # changes the number no longer applies and the bench reports null.
-MEASURED_TRAFFIC = {"86f2af96b916765d": 248780544}
+MEASURED_TRAFFIC = {"b7634f37e38a8462": 248863488}
 DEFAULT_WORKLOAD = "gqa_decode"
 FALLBACK_HBM_GBS = 6650.0
 N_POOLS = 3

@@ -1367,6 +1367,39 @@ bool encode_kv_map(CUtensorMap *m, const void *base, int D, int Hkv, long long p
   return r == CUDA_SUCCESS;
 }
 
+// The K and V maps of a call, from a small per-thread cache: a decode loop
+// calls with the same cache buffers step after step, and encoding the two
+// maps is a noticeable part of the host time of a short call.  The key is
+// every input of the encoding, so a hit is always the map the call needs.
+bool kv_maps(TmapPair *tm, const void *k, const void *v, int D, int Hkv, long long pool_tokens, int box_tokens,
+             bool bf16) {
+  struct Entry {
+    const void *k, *v;
+    long long pool_tokens;
+    int D, Hkv, box_tokens;
+    bool bf16, used;
+    TmapPair tm;
+  };
+  constexpr int kEntries = 4;
+  thread_local Entry cache[kEntries] = {};
+  thread_local int next = 0;
+  for (int i = 0; i < kEntries; ++i) {
+    const Entry &e = cache[i];
+    if (e.used && e.k == k && e.v == v && e.pool_tokens == pool_tokens && e.D == D && e.Hkv == Hkv &&
+        e.box_tokens == box_tokens && e.bf16 == bf16) {
+      *tm = e.tm;
+      return true;
+    }
+  }
+  if (!encode_kv_map(&tm->k, k, D, Hkv, pool_tokens, box_tokens, bf16) ||
+      !encode_kv_map(&tm->v, v, D, Hkv, pool_tokens, box_tokens, bf16))
+    return false;
+  Entry &e = cache[next];
+  next = (next + 1) % kEntries;
+  e = Entry{k, v, pool_tokens, D, Hkv, box_tokens, bf16, true, *tm};
+  return true;
+}
+
 template <int D, bool kBf16, bool kAppend>
 cudaError_t prepare_split_kernel(int device) {
   static std::mutex mu;
@@ -1441,9 +1474,7 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
 
   TmapPair tm;
   const long long pool_tokens = (long long)(a.contiguous ? p.B : p.num_pages) * p.page_size;
-  if (!encode_kv_map(&tm.k, L.k_cache, D, p.Hkv, pool_tokens, a.box_tokens, kBf16) ||
-      !encode_kv_map(&tm.v, L.v_cache, D, p.Hkv, pool_tokens, a.box_tokens, kBf16))
-    return MXA_ERR_CUDA;
+  if (!kv_maps(&tm, L.k_cache, L.v_cache, D, p.Hkv, pool_tokens, a.box_tokens, kBf16)) return MXA_ERR_CUDA;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)plan.grid);

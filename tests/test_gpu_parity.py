@@ -281,3 +281,30 @@ def test_combine_matches_exact_merge(dtype):
     torch.cuda.synchronize()
     assert_out_close(out.cpu(), ro.reshape(B, q_len, Hq, D), dtype)
     assert_lse_close(lse_out.cpu(), rl.reshape(B, q_len, Hq).transpose(0, 2, 1))
+
+
+# --------------------------------------------------------------------------
+# CUDA graphs: a decode step captured once and replayed
+# --------------------------------------------------------------------------
+
+def test_decode_replays_in_a_cuda_graph():
+    inp, ref, dev = full(1)
+    q, k, v, bt, sl = dev
+    w = inp.w
+    prep = mxa.prepare(q, k, bt, max_seqlen_k=inp.max_seqlen_k)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=q.device)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):  # first call outside the capture (kernel attributes, maps)
+        mxa.decode(q, k, v, bt, sl, scale=w.scale, causal=w.causal, prepared=prep, out=out, lse=lse)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        mxa.decode(q, k, v, bt, sl, scale=w.scale, causal=w.causal, prepared=prep, out=out, lse=lse)
+    out.zero_()
+    lse.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert mxa.mxa_device_error(True) == mxa.MXA_OK
+    check(inp, out.cpu(), lse.cpu(), ref)
