@@ -81,6 +81,10 @@ CASES = [
     # head_dim 64, fp16, groups of 2, small pages; rows whose cache was empty
     dict(B=6, q_len=2, Hq=16, Hkv=8, D=64, dtype="f16", page_size=8, causal=True,
          lengths="list:2,3,17,130,2,900"),
+    # 4 draft tokens x 8 query heads = 32 packed rows: two row tiles per KV head,
+    # whose units both write the new tokens (the same bytes) before reading them
+    dict(B=3, q_len=4, Hq=16, Hkv=2, D=128, dtype="bf16", page_size=16, causal=True,
+         lengths="list:5,300,2049"),
 ]
 
 
