@@ -235,7 +235,7 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(tot_t / args.steps * 1e3, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, algorithmic_bytes(inp), world),
+        "config": dict(workload_config(w, algorithmic_bytes(inp), world), append=False),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": omp_threads(),
                          "kind": "oracle", "sample": f"first {rows} of {w.B} rows per step"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
