@@ -81,6 +81,46 @@ def decode(q, k_cache, v_cache, block_table, cache_seqlens, *, Hkv: int,
     return out, lse
 
 
+def decode_varlen(q, cu_seqlens_q, k_cache, v_cache, block_table, cache_seqlens, *, Hkv: int,
+                  page_size: int, dtype: str, scale: float, causal: bool) -> Tuple[np.ndarray, np.ndarray]:
+    """Exact attention for rows with their own number of queries, in fp64.
+
+    The packed-query layout of a varlen call: row b's queries are
+    q[cu_seqlens_q[b] : cu_seqlens_q[b + 1]] ("MXFlashAttn 1.4.0",
+    flash_attn_varlen_func; "MixedQuantSparseFlashMlaMetadata 算子解析",
+    参数说明: cu_seqlens of B + 1 entries, starting at 0, non-decreasing).  Each
+    row is the plain decode of decode() with its own q_len_b; with causal
+    the row's queries are its last q_len_b cache entries (query t sees the
+    first L_b - q_len_b + t + 1 keys).
+
+    q [total_q, Hq, D]; caches and block_table as for decode().
+    Returns (out [total_q, Hq, D] float64, lse [Hq, total_q] float64).
+    """
+    qb = _bits(q)
+    total_q, Hq, D = qb.shape
+    cu = np.asarray(cu_seqlens_q, dtype=np.int64)
+    L = np.asarray(cache_seqlens, dtype=np.int32)
+    if cu.ndim != 1 or cu[0] != 0 or cu[-1] != total_q or (np.diff(cu) < 0).any():
+        raise ValueError("cu_seqlens_q: B + 1 non-decreasing offsets from 0 to total_q")
+    out = np.zeros((total_q, Hq, D), dtype=np.float64)
+    lse = np.zeros((Hq, total_q), dtype=np.float64)
+    bt = None if block_table is None else np.asarray(block_table, dtype=np.int32)
+    for b in range(cu.size - 1):
+        q0, q1 = int(cu[b]), int(cu[b + 1])
+        if q1 == q0:
+            continue
+        row_bt = None if bt is None else bt[b:b + 1]
+        if bt is None:  # contiguous cache: row b only
+            kc, vc = _bits(k_cache)[b:b + 1], _bits(v_cache)[b:b + 1]
+        else:
+            kc, vc = _bits(k_cache), _bits(v_cache)
+        o, l = decode(qb[None, q0:q1], kc, vc, row_bt, L[b:b + 1], Hkv=Hkv, page_size=page_size,
+                      dtype=dtype, scale=scale, causal=causal)
+        out[q0:q1] = o[0]
+        lse[:, q0:q1] = l[0]
+    return out, lse
+
+
 def append_kv(k_cache, v_cache, k_new, v_new, block_table, cache_seqlens, *, page_size: int):
     """Write each row's new tokens into copies of the caches; return the copies.
 
