@@ -31,6 +31,8 @@ mxa_status_t check_shape(const mxa_decode_params_t *p) {
   const long long units = (long long)p->B * p->Hkv * RT;
   const long long blocks = units * ceil_div_ll(p->max_seqlen_k, T);
   if (units > INT32_MAX || blocks > INT32_MAX) return MXA_ERR_UNSUPPORTED;
+  // the balanced prologue sums every row's blocks plus its unit cost in 32 bits
+  if (blocks + (long long)p->B * kMaxUnitCost > INT32_MAX) return MXA_ERR_UNSUPPORTED;
   if ((long long)p->num_pages * p->page_size > INT32_MAX) return MXA_ERR_UNSUPPORTED;  // TMA coordinates
   return MXA_OK;
 }

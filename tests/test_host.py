@@ -223,6 +223,19 @@ def test_append_refuses_bad_arguments_before_launch():
                                           None) == MXA_OK  # nothing to do for B = 0 (paged layout)
 
 
+def test_shapes_whose_position_sums_overflow_are_refused():
+    # B rows x max KV blocks fits 32 bits, but not once every row's unit cost
+    # (up to 64 blocks) is added: the balanced prologue's sums would overflow
+    ok = params(B=1000, Hq=1, Hkv=1, page_size=64, num_pages=16, max_pages_per_seq=2147000,
+                max_seqlen_k=2147000 * 64)
+    assert mxa.mxa_plan(ok, 0, sm_count=148).schedule in (MXA_SCHED_BALANCED, mxa.MXA_SCHED_UNIFORM)
+    big = params(B=1000, Hq=1, Hkv=1, page_size=64, num_pages=16, max_pages_per_seq=2147483,
+                 max_seqlen_k=2147483 * 64)
+    with pytest.raises(mxa.MxaError) as e:
+        mxa.mxa_plan(big, 0, sm_count=148)
+    assert e.value.code == mxa.MXA_ERR_UNSUPPORTED
+
+
 def test_combine_refuses_bad_arguments():
     f = lambda x: None if x is None else ctypes.c_void_p(x * 4096)
     c = mxa._lib.mxa_combine
