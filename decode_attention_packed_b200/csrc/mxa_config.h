@@ -46,7 +46,7 @@ struct SegmentDesc {
   int c_first;           // first CTA holding a piece of the unit
   int n_pieces;          // CTAs holding pieces of the unit
   int last;              // 1 if no segment follows in this CTA
-  int pad[2];
+  int q0, qn;            // row b's first packed query token and its query count
 };
 
 // What the math warps hand to the epilogue warp at the end of a segment:

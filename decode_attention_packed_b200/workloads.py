@@ -178,6 +178,18 @@ def make_inputs(w: Workload, seed: Optional[int] = None,
                   max_seqlen_k=max_seqlen_k)
 
 
+def make_varlen_queries(q_lens, Hq: int, D: int, dtype: str, seed: int):
+    """Queries of rows with their own query counts, packed: q [total_q, Hq, D]
+    (N(0, 1) rounded to `dtype`) and the offsets cu [B + 1] int32 (0, then the
+    running totals of q_lens)."""
+    rng = np.random.default_rng(seed)
+    ql = np.asarray(q_lens, dtype=np.int64)
+    assert ql.ndim == 1 and (ql >= 0).all()
+    cu = np.concatenate([[0], np.cumsum(ql)]).astype(np.int32)
+    q = rng.standard_normal((int(cu[-1]), Hq, D), dtype=np.float32)
+    return _round(q, dtype), torch.from_numpy(cu)
+
+
 def small_variant(w: Workload, **changes) -> Workload:
     """The same recipe with some fields changed (used for parity cases the
     oracle finishes in seconds)."""

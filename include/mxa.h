@@ -231,6 +231,34 @@ MXA_API mxa_status_t mxa_decode_fwd_append(const void *q, void *k_cache, void *v
                                            float scale, int causal, const mxa_plan_t *plan, void *workspace,
                                            size_t workspace_bytes, void *out, float *lse, void *stream);
 
+/* Decode rows that each have their own number of queries: the packed
+ * (varlen) layout of flash_attn_varlen_func ("MXFlashAttn 1.4.0", its API
+ * list), with the cu_seqlens_q offsets defined in
+ * "MixedQuantSparseFlashMlaMetadata 算子解析" (参数说明).
+ *   q            : device [total_q, Hq, D] dtype; row b's queries are
+ *                  q[cu_seqlens_q[b] .. cu_seqlens_q[b + 1] - 1]
+ *   cu_seqlens_q : device [B + 1] int32, read only: 0 = cu[0] <= cu[1] <= ...
+ *                  <= cu[B] = total_q
+ *   total_q      : packed query tokens (>= 0)
+ *   params->q_len: the largest per-row query count (max_seqlen_q); it sizes
+ *                  the plan (mxa_plan with these params) and the workspace
+ *   out          : device [total_q, Hq, D] dtype (written in full)
+ *   lse          : device [Hq, total_q] float32, or NULL to skip
+ * Row b with q_b = cu[b+1] - cu[b] queries: non-causal, every query sees L_b
+ * keys; causal, query t sees the first L_b - q_b + t + 1 (its queries are
+ * the row's last q_b cache entries).  A row with q_b = 0 writes nothing.
+ * Offsets are read on the device and not checked there against these rules:
+ * out-of-range values are clamped into [0, total_q] and a row's count to
+ * params->q_len, so that no access leaves the buffers, but the result of
+ * such a call is unspecified.  Other arguments and errors as
+ * mxa_decode_fwd_with_plan; MXA_ERR_INVALID_ARG for a NULL or misaligned
+ * cu_seqlens_q or total_q < 0. */
+MXA_API mxa_status_t mxa_decode_fwd_varlen(const void *q, const int32_t *cu_seqlens_q, int total_q,
+                                   const void *k_cache, const void *v_cache, const int32_t *block_table,
+                                   const int32_t *cache_seqlens, const mxa_decode_params_t *params,
+                                   float scale, int causal, const mxa_plan_t *plan, void *workspace,
+                                   size_t workspace_bytes, void *out, float *lse, void *stream);
+
 /* Decode without any device allocation, for callers that cannot allocate.
  * (An addition of this library; the source pages have no counterpart.)
  *
