@@ -324,7 +324,8 @@ mxa_status_t mxa_device_error(int reset) {
   int flags = 0;
   mxa_status_t st = read_device_error(reset, &flags);
   if (st != MXA_OK) return st;
-  return flags ? MXA_ERR_TIMEOUT : MXA_OK;
+  if (flags & ~kErrBadPage) return MXA_ERR_TIMEOUT;
+  return flags ? MXA_ERR_INVALID_ARG : MXA_OK;  // an appended token's page id was outside the pool
 }
 
 }  // extern "C"

@@ -18,6 +18,13 @@ constexpr int kMaxThreadsPerSm = 2048;
 constexpr int kMaxBalancedRows = 12288;                 // balanced schedule scans B rows in smem
 constexpr int kMaxUnitCost = 64;
 
+// Device-side failure record (bit flags), read back by mxa_device_error():
+// bounded waits that ran out, a misaligned shared-memory base, and appended
+// tokens whose page id lay outside the pool (not written).
+enum : int {
+  kErrWaitFull = 1, kErrWaitEmpty = 2, kErrWaitQ = 4, kErrAlign = 8, kErrDrain = 16, kErrBadPage = 32
+};
+
 // Fixed cost of a unit in the balanced schedule, in KV blocks: the work a
 // unit needs besides streaming its keys (the cross-warp merge, the output
 // staging and stores, the arrival and merge of a split unit) grows with its

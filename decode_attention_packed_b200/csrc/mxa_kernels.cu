@@ -438,7 +438,12 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
         const int idx = p / ps - w.base;
         const int va = __shfl_sync(0xffffffffu, w.wa, idx & 31);
         const int vb = __shfl_sync(0xffffffffu, w.wb, idx & 31);
-        token = (long long)(idx < 32 ? va : vb) * ps + p % ps;
+        const int page = idx < 32 ? va : vb;  // the same in every lane
+        if (page < 0 || page >= a.num_pages) {  // not a page of the pool: skip the token, report it
+          if (lane == 0) atomicOr(&g_mxa_err, kErrBadPage);
+          continue;
+        }
+        token = (long long)page * ps + p % ps;
       }
       if (lane < 2 * CW) {
         const bool is_v = lane >= CW;
@@ -1525,6 +1530,7 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
   a.RT = (a.M + kRowsPerTile - 1) / kRowsPerTile;
   a.contiguous = L.block_table == nullptr;
   a.page_size = p.page_size;
+  a.num_pages = p.num_pages;
   a.mpps = p.max_pages_per_seq;
   a.max_seqlen_k = p.max_seqlen_k;
   a.box_tokens = a.contiguous ? T : (p.page_size % T == 0 ? T : p.page_size);

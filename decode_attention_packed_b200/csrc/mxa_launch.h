@@ -30,6 +30,7 @@ struct DecodeArgs {
   int B, q_len, Hq, Hkv, G, M, RT;  // varlen: q_len bounds every row's query count
   int total_q;                 // varlen: packed query tokens
   int page_size;               // slots per page (row capacity when contiguous)
+  int num_pages;               // pages in the pool (paged)
   int mpps;                    // block-table row stride
   int contiguous;
   int max_seqlen_k;

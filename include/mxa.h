@@ -220,7 +220,9 @@ MXA_API mxa_status_t mxa_decode_fwd_with_plan(const void *q, const void *k_cache
  * Every query row then attends to the first L_b + q_len keys; with causal = 1
  * query t sees the first L_b + t + 1.  params->max_seqlen_k bounds L_b + q_len
  * (tokens that would land at or past it, or past the row's block-table
- * width, are not written).  The plan is that of mxa_plan for `params`.  One
+ * width, are not written; nor is a token whose page id lies outside
+ * [0, num_pages): mxa_device_error then reports MXA_ERR_INVALID_ARG).  The
+ * plan is that of mxa_plan for `params`.  One
  * kernel runs on `stream`: the CTA that streams the block holding an
  * appended token writes the token into the cache (for its KV head) and then
  * loads the block, so each token is written before it is read.
@@ -304,9 +306,11 @@ MXA_API mxa_status_t mxa_combine(const float *o_part, const float *lse_part, int
                          void *stream);
 
 /* Synchronise the current device and report whether any kernel of this
- * library recorded a device-side failure (a bounded wait that ran out) since
- * the last reset: MXA_OK or MXA_ERR_TIMEOUT (MXA_ERR_CUDA if the device or
- * the synchronisation itself failed).  reset != 0 clears the record. */
+ * library recorded a device-side failure since the last reset: MXA_OK;
+ * MXA_ERR_TIMEOUT if a bounded wait ran out; else MXA_ERR_INVALID_ARG if an
+ * appended token's page id lay outside [0, num_pages) (the token was not
+ * written); MXA_ERR_CUDA if the device or the synchronisation itself failed.
+ * reset != 0 clears the record. */
 MXA_API mxa_status_t mxa_device_error(int reset);
 
 #ifdef __cplusplus
