@@ -337,6 +337,22 @@ def main():
     dev_s = max_over_ranks(e0.elapsed_time(e1) / 1e3)
     assert mxa.mxa_device_error(True) == mxa.MXA_OK, "device-side wait ran out during the bench"
 
+    # ---- spread of single calls: each call between its own pair of events
+    # (so neighbouring calls do not overlap it), after the timed region ----
+    n_each = max(1, min(args.steps, 2000))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_each + 1)]
+    barrier()
+    ev[0].record(stream)
+    for i in range(n_each):
+        call(i)
+        ev[i + 1].record(stream)
+    barrier()
+    each_us = sorted(ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(n_each))
+    pct = lambda f: round(each_us[min(n_each - 1, int(f * n_each))], 3)
+    per_call = {"p10": pct(0.10), "p50": pct(0.50), "p90": pct(0.90), "n": n_each, "unit": "us",
+                "how": "each call between its own events, back to back; the headline value is the mean "
+                       "over the timed region"}
+
     # ---- end to end through the C ABI: every step copies its inputs from
     # pinned host memory (query, block table, lengths; the KV cache lives on
     # the device) and reads its result back (output and LSE).  As in a
@@ -420,6 +436,7 @@ def main():
         "warmup": args.warmup,
         "ms_per_step": round(dev_s / args.steps * 1e3, 5),
         "us_per_call": round(per_call_s * 1e6, 3),
+        "per_call_us": per_call,
         "kv_frac_of_hbm_peak": round(kv_gbs / peak, 4),
         "higher_is_better": True,
         "scaling": "weak",

@@ -76,7 +76,15 @@ WORKLOADS = [
              page_size=16, causal=False, lengths="loguniform:1:16384", k_scale=3.0, seed=1004),
 ]
 
-BY_NAME = {w.name: w for w in WORKLOADS}
+# Other readings of the workloads above, benchmarked for context only: the
+# speculative step with every row at 8192 keys (the spec/MTP lengths read as
+# "all rows 8192" instead of the cycle through the non-power-of-two lengths).
+CONTEXT_WORKLOADS = [
+    Workload("spec_mtp_small_q_all8192", B=16, q_len=4, Hq=32, Hkv=8, D=128, dtype="bf16",
+             page_size=64, causal=True, lengths="const:8192", seed=1012),
+]
+
+BY_NAME = {w.name: w for w in WORKLOADS + CONTEXT_WORKLOADS}
 
 
 def workload(name_or_index) -> Workload:
