@@ -19,8 +19,9 @@ constexpr int kMaxBalancedRows = 12288;                 // balanced schedule sca
 constexpr int kMaxUnitCost = 64;
 
 // Device-side failure record (bit flags), read back by mxa_device_error():
-// bounded waits that ran out, a misaligned shared-memory base, and appended
-// tokens whose page id lay outside the pool (not written).
+// bounded waits that ran out, a misaligned shared-memory base, and
+// block-table entries outside the pool (read as zeros; appended tokens there
+// not written).
 enum : int {
   kErrWaitFull = 1, kErrWaitEmpty = 2, kErrWaitQ = 4, kErrAlign = 8, kErrDrain = 16, kErrBadPage = 32
 };

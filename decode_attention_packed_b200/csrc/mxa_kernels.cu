@@ -458,6 +458,7 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
   int it = 0;     // KV stages issued
   int seg_k = 0;  // segments published
   bool ok = true;
+  bool bad_page = false;  // a block-table entry outside [0, num_pages) was met
   if (more()) {
     SegmentDesc seg = take();
     seg.last = more() ? 0 : 1;
@@ -518,6 +519,10 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
             const int va = __shfl_sync(0xffffffffu, win.wa, src);
             const int vb = __shfl_sync(0xffffffffu, win.wb, src);
             page = idx < 32 ? va : vb;
+            if (page < 0 || page >= a.num_pages) {  // not a page of the pool: read as zeros, reported
+              bad_page |= op < n_ops;
+              page = -1;  // rows [-page_size, 0): outside the map, so the box is filled with zeros
+            }
           }
           if (op < n_ops) {
             const int row = a.contiguous ? seg.b * ps + tok : page * ps + tok % ps;
@@ -566,6 +571,7 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
     }
   }
 
+  if (__any_sync(0xffffffffu, bad_page) && lane == 0) atomicOr(&g_mxa_err, kErrBadPage);
   if (ok && warp_wait_bounded(qempty, (seg_k & 1) ^ 1, &g_mxa_err, kErrWaitQ, lane)) {
     if (lane == 0) {  // end-of-work marker for the math warps
       SegmentDesc d{};

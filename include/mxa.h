@@ -83,6 +83,9 @@ typedef enum { MXA_SCHED_UNIFORM = 0, MXA_SCHED_BALANCED = 1 } mxa_schedule_t;
  *                [B, page_size, Hkv, D]             dtype   (contiguous: block_table == NULL,
  *                                                            num_pages == B, page_size = row capacity)
  *   block_table  [B, max_pages_per_seq] int32: page id of logical page p of row b
+ *                (an id outside [0, num_pages) is never dereferenced: its keys
+ *                and values read as zeros, and mxa_device_error reports
+ *                MXA_ERR_INVALID_ARG)
  *   cache_seqlens[B] int32: number of valid keys L_b, 0 <= L_b <= max_seqlen_k
  *   out          [B, q_len, Hq, D]                 dtype
  *   lse          [B, Hq, q_len]                    float32, natural log
@@ -307,9 +310,10 @@ MXA_API mxa_status_t mxa_combine(const float *o_part, const float *lse_part, int
 
 /* Synchronise the current device and report whether any kernel of this
  * library recorded a device-side failure since the last reset: MXA_OK;
- * MXA_ERR_TIMEOUT if a bounded wait ran out; else MXA_ERR_INVALID_ARG if an
- * appended token's page id lay outside [0, num_pages) (the token was not
- * written); MXA_ERR_CUDA if the device or the synchronisation itself failed.
+ * MXA_ERR_TIMEOUT if a bounded wait ran out; else MXA_ERR_INVALID_ARG if a
+ * block-table entry that a kernel used lay outside [0, num_pages) (its keys
+ * read as zeros; an appended token there was not written); MXA_ERR_CUDA if
+ * the device or the synchronisation itself failed.
  * reset != 0 clears the record. */
 MXA_API mxa_status_t mxa_device_error(int reset);
 
