@@ -31,7 +31,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from decode_attention_packed_b200.workloads import WORKLOADS, make_inputs, workload  # noqa: E402
+from decode_attention_packed_b200.workloads import WORKLOADS, make_inputs, make_varlen_queries, workload  # noqa: E402
 
 METRIC = "decode-attn µs/call and KV-read GB/s as % of B200 HBM peak (1 GPU)"
 
@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--append", action="store_true",
                     help="each step also appends the step's q_len new tokens per row to the cache "
                          "(mxa_decode_fwd_append) before attending")
+    ap.add_argument("--varlen", action="store_true",
+                    help="rows have their own query counts, drawn (seeded) from 1..q_len, packed with "
+                         "cu_seqlens_q (mxa_decode_fwd_varlen)")
     return ap.parse_args()
 
 
@@ -255,6 +258,8 @@ def main():
 
     w = workload(args.workload)
     inp = shard_inputs(w, rank)
+    if args.append and args.varlen:
+        raise SystemExit("--append and --varlen do not combine")
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     q = inp.q.to(dev)
@@ -265,8 +270,15 @@ def main():
         pools.append((pools[0][0].clone(), pools[0][1].clone()))
     splits = w.num_splits if args.num_splits is None else args.num_splits
     prep = mxa.prepare(q, pools[0][0], bt, max_seqlen_k=inp.max_seqlen_k, num_splits=splits)
+    cu = hcu = None
+    if args.varlen:  # the plan above is for q_len queries per row, which bounds every row's count
+        q_lens = np.random.default_rng(w.seed + 77).integers(1, w.q_len + 1, size=w.B)
+        hqv, hcu = make_varlen_queries(q_lens, w.Hq, w.D, w.dtype, w.seed + 78)
+        q, cu = hqv.to(dev), hcu.to(dev)
+        hcu = hcu.pin_memory()
     out = torch.empty_like(q)
-    lse = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=dev)
+    lse = (torch.empty((w.Hq, q.shape[0]), dtype=torch.float32, device=dev) if args.varlen
+           else torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=dev))
     nbytes = algorithmic_bytes(inp)
     if args.append:  # the new tokens are read and written once more
         nbytes["total"] += 2 * 2 * w.B * w.q_len * w.Hkv * w.D * inp.q.element_size()
@@ -279,14 +291,20 @@ def main():
         k_new = torch.randn((w.B, w.q_len, w.Hkv, w.D), device=dev).to(q.dtype)
         v_new = torch.randn_like(k_new)
 
-    def call(i):
+    def run(i, q, cu, bt, sl, out, lse):
         k, v = pools[i % N_POOLS]
         if args.append:
-            mxa.mxa_decode_fwd_append(q, k, v, k_new, v_new, bt, sl_before, prep.params, w.scale, w.causal,
+            mxa.mxa_decode_fwd_append(q, k, v, k_new, v_new, bt, sl, prep.params, w.scale, w.causal,
                                       prep.plan, prep.workspace, out, lse, stream)
+        elif args.varlen:
+            mxa.mxa_decode_fwd_varlen(q, cu, k, v, bt, sl, prep.params, w.scale, w.causal, prep.plan,
+                                      prep.workspace, out, lse, stream)
         else:
             mxa.mxa_decode_fwd_with_plan(q, k, v, bt, sl, prep.params, w.scale, w.causal, prep.plan,
                                          prep.workspace, out, lse, stream)
+
+    def call(i):
+        run(i, q, cu, bt, sl_before if args.append else sl, out, lse)
 
     def barrier():
         if world > 1:
@@ -319,16 +337,33 @@ def main():
     dev_s = max_over_ranks(e0.elapsed_time(e1) / 1e3)
     assert mxa.mxa_device_error(True) == mxa.MXA_OK, "device-side wait ran out during the bench"
 
+    # ---- spread of single calls: each call between its own pair of events
+    # (so neighbouring calls do not overlap it), after the timed region ----
+    n_each = max(1, min(args.steps, 2000))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_each + 1)]
+    barrier()
+    ev[0].record(stream)
+    for i in range(n_each):
+        call(i)
+        ev[i + 1].record(stream)
+    barrier()
+    each_us = sorted(ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(n_each))
+    pct = lambda f: round(each_us[min(n_each - 1, int(f * n_each))], 3)
+    per_call = {"p10": pct(0.10), "p50": pct(0.50), "p90": pct(0.90), "n": n_each, "unit": "us",
+                "how": "each call between its own events, back to back; the headline value is the mean "
+                       "over the timed region"}
+
     # ---- end to end through the C ABI: every step copies its inputs from
     # pinned host memory (query, block table, lengths; the KV cache lives on
     # the device) and reads its result back (output and LSE).  As in a
     # serving loop the copies run on their own streams and overlap the
     # previous and next steps' kernels: inputs and outputs are double
     # buffered, and events order each buffer's copy-in, decode and copy-out.
-    hq = inp.q.pin_memory()
+    hq = (hqv if args.varlen else inp.q).pin_memory()
     hbt = None if inp.block_table is None else inp.block_table.pin_memory()
     hsl = ((inp.cache_seqlens - w.q_len).clamp(min=0) if args.append else inp.cache_seqlens).pin_memory()
-    h2d = hq.numel() * hq.element_size() + hsl.numel() * 4 + (0 if hbt is None else hbt.numel() * 4)
+    h2d = (hq.numel() * hq.element_size() + hsl.numel() * 4 + (0 if hbt is None else hbt.numel() * 4)
+           + (0 if hcu is None else hcu.numel() * 4))
     d2h = out.numel() * out.element_size() + lse.numel() * 4
     e2e_steps = max(1, min(args.steps, 2000))
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -336,6 +371,7 @@ def main():
     for _ in range(2):
         slots.append(dict(
             q=torch.empty_like(q), sl=torch.empty_like(sl), bt=None if bt is None else torch.empty_like(bt),
+            cu=None if cu is None else torch.empty_like(cu),
             out=torch.empty_like(out), lse=torch.empty_like(lse),
             hout=torch.empty(out.shape, dtype=out.dtype, pin_memory=True),
             hlse=torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True),
@@ -352,16 +388,12 @@ def main():
             sd["sl"].copy_(hsl, non_blocking=True)
             if hbt is not None:
                 sd["bt"].copy_(hbt, non_blocking=True)
+            if hcu is not None:
+                sd["cu"].copy_(hcu, non_blocking=True)
             sd["copied"].record(s_in)
         stream.wait_event(sd["copied"])
         stream.wait_event(sd["read"])  # the read-back two steps back is done with these outputs
-        k, v = pools[i % N_POOLS]
-        if args.append:
-            mxa.mxa_decode_fwd_append(sd["q"], k, v, k_new, v_new, sd["bt"], sd["sl"], prep.params, w.scale,
-                                      w.causal, prep.plan, prep.workspace, sd["out"], sd["lse"], stream)
-        else:
-            mxa.mxa_decode_fwd_with_plan(sd["q"], k, v, sd["bt"], sd["sl"], prep.params, w.scale, w.causal,
-                                         prep.plan, prep.workspace, sd["out"], sd["lse"], stream)
+        run(i, sd["q"], sd["cu"], sd["bt"], sd["sl"], sd["out"], sd["lse"])
         sd["decoded"].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(sd["decoded"])
@@ -404,18 +436,21 @@ def main():
         "warmup": args.warmup,
         "ms_per_step": round(dev_s / args.steps * 1e3, 5),
         "us_per_call": round(per_call_s * 1e6, 3),
+        "per_call_us": per_call,
         "kv_frac_of_hbm_peak": round(kv_gbs / peak, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic",
-        "config": dict(workload_config(w, nbytes, world), append=bool(args.append)),
+        "config": dict(workload_config(w, nbytes, world), append=bool(args.append),
+                       **({"varlen": {"q_lens": "U{1..%d} per row, seeded" % w.q_len,
+                                      "total_q": int(q.shape[0])}} if args.varlen else {})),
         "plan": prep.plan.as_dict(),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "traffic": MEASURED_TRAFFIC.get(kernel_source_hash())
-                     if w.name == DEFAULT_WORKLOAD and not args.append else None,
+                     if w.name == DEFAULT_WORKLOAD and not (args.append or args.varlen) else None,
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                      else "fallback 6.65 TB/s",
                      "kernel": "mxa_split_kernel (one launch per call; split units merged inside)"},

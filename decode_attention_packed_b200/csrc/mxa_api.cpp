@@ -111,6 +111,8 @@ mxa_status_t prepare_decode(const void *q, const void *k_cache, const void *v_ca
   L.causal = causal;
   L.len_add = 0;
   L.k_new = L.v_new = nullptr;
+  L.cu_q = nullptr;
+  L.total_q = 0;
   return MXA_OK;
 }
 
@@ -270,6 +272,30 @@ mxa_status_t mxa_decode_fwd_append(const void *q, void *k_cache, void *v_cache, 
   return launch_decode(L, static_cast<cudaStream_t>(stream));
 }
 
+mxa_status_t mxa_decode_fwd_varlen(const void *q, const int32_t *cu_seqlens_q, int total_q, const void *k_cache,
+                                   const void *v_cache, const int32_t *block_table, const int32_t *cache_seqlens,
+                                   const mxa_decode_params_t *p, float scale, int causal, const mxa_plan_t *plan,
+                                   void *workspace, size_t workspace_bytes, void *out, float *lse, void *stream) {
+  if (p == nullptr || total_q < 0) return MXA_ERR_INVALID_ARG;
+  if (p->B > 0 && (cu_seqlens_q == nullptr || !aligned(cu_seqlens_q, 4))) return MXA_ERR_INVALID_ARG;
+  if (total_q == 0) {  // no query: nothing is written
+    mxa_status_t st = check_shape(p);
+    return st != MXA_OK ? st : check_layout(p, block_table == nullptr);
+  }
+  DecodeLaunch L;
+  mxa_status_t st = prepare_decode(q, k_cache, v_cache, block_table, cache_seqlens, p, scale, causal, plan,
+                                   workspace, workspace_bytes, out, lse, &L);
+  if (st != MXA_OK || p->B == 0) return st;
+  // the balanced prologue sums positions of one KV head's tiles per row in 32 bits
+  const long long G = p->Hq / p->Hkv;
+  const long long RT = ceil_div_ll((long long)p->q_len * G, kRowsPerTile);
+  const long long row_max = RT * (ceil_div_ll(p->max_seqlen_k, block_tokens(p->D)) + L.plan.unit_cost);
+  if (L.plan.schedule == MXA_SCHED_BALANCED && (long long)p->B * row_max > INT32_MAX) return MXA_ERR_UNSUPPORTED;
+  L.cu_q = cu_seqlens_q;
+  L.total_q = total_q;
+  return launch_decode(L, static_cast<cudaStream_t>(stream));
+}
+
 mxa_status_t mxa_decode_fwd(const void *q, const void *k_cache, const void *v_cache,
                             const int32_t *block_table, const int32_t *cache_seqlens,
                             const mxa_decode_params_t *p, float scale, int causal, int num_splits,
@@ -298,7 +324,8 @@ mxa_status_t mxa_device_error(int reset) {
   int flags = 0;
   mxa_status_t st = read_device_error(reset, &flags);
   if (st != MXA_OK) return st;
-  return flags ? MXA_ERR_TIMEOUT : MXA_OK;
+  if (flags & ~kErrBadPage) return MXA_ERR_TIMEOUT;
+  return flags ? MXA_ERR_INVALID_ARG : MXA_OK;  // an appended token's page id was outside the pool
 }
 
 }  // extern "C"

@@ -18,6 +18,14 @@ constexpr int kMaxThreadsPerSm = 2048;
 constexpr int kMaxBalancedRows = 12288;                 // balanced schedule scans B rows in smem
 constexpr int kMaxUnitCost = 64;
 
+// Device-side failure record (bit flags), read back by mxa_device_error():
+// bounded waits that ran out, a misaligned shared-memory base, and
+// block-table entries outside the pool (read as zeros; appended tokens there
+// not written).
+enum : int {
+  kErrWaitFull = 1, kErrWaitEmpty = 2, kErrWaitQ = 4, kErrAlign = 8, kErrDrain = 16, kErrBadPage = 32
+};
+
 // Fixed cost of a unit in the balanced schedule, in KV blocks: the work a
 // unit needs besides streaming its keys (the cross-warp merge, the output
 // staging and stores, the arrival and merge of a split unit) grows with its
@@ -46,7 +54,7 @@ struct SegmentDesc {
   int c_first;           // first CTA holding a piece of the unit
   int n_pieces;          // CTAs holding pieces of the unit
   int last;              // 1 if no segment follows in this CTA
-  int pad[2];
+  int q0, qn;            // row b's first packed query token and its query count
 };
 
 // What the math warps hand to the epilogue warp at the end of a segment:

@@ -8,10 +8,9 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-namespace mxa {
+#include "mxa_config.h"
 
-// Device-side failure record (bit flags), read back by mxa_device_error().
-enum : int { kErrWaitFull = 1, kErrWaitEmpty = 2, kErrWaitQ = 4, kErrAlign = 8, kErrDrain = 16 };
+namespace mxa {
 
 // A bounded wait gives up after this long and records a failure instead of
 // spinning forever.

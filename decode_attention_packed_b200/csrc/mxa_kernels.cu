@@ -78,27 +78,71 @@ struct Cursor {
   long long per_cta;  // positions per CTA range (balanced schedule)
   int L, nb;          // length and blocks of row b
   int L_next;         // prefetched length of row b + 1
+  int rtb;            // row tiles of row b: its units are hr < Hkv * rtb
+  int q0, qn;         // row b's queries: first packed token, count
+  int q0_next, qn_next;  // prefetched queries of row b + 1 (per-row queries only)
 };
 
-template <int D>
+// Queries of batch row b: its first packed token q0 and its count qn.  With
+// per-row offsets the offsets read are clamped, so that every index stays in
+// [0, total_q) and no row holds more than q_len queries (the bound its tiles
+// and arrival counters were sized for).
+template <bool kVarlen>
+__device__ __forceinline__ void row_queries(const DecodeArgs &a, int b, int &q0, int &qn) {
+  if constexpr (kVarlen) {
+    const int s = min(max(a.cu_q[b], 0), a.total_q);
+    const int e = min(max(a.cu_q[b + 1], s), a.total_q);
+    q0 = s;
+    qn = min(e - s, a.q_len);
+  } else {
+    q0 = b * a.q_len;
+    qn = a.q_len;
+  }
+}
+
+// Row tiles of a row with qn queries, and the packed rows of its tile rt.
+__device__ __forceinline__ int row_tiles(const DecodeArgs &a, int qn) {
+  return (qn * a.G + kRowsPerTile - 1) / kRowsPerTile;
+}
+__device__ __forceinline__ int tile_rows(const DecodeArgs &a, int qn, int rt) {
+  return min(kRowsPerTile, qn * a.G - rt * kRowsPerTile);
+}
+
+// Index of the LSE of query t of row b (first packed token q0), head hq:
+// [B, Hq, q_len], or [Hq, total_q] with per-row offsets.
+__device__ __forceinline__ size_t lse_index(const DecodeArgs &a, int b, int q0, int hq, int t) {
+  return a.cu_q != nullptr ? (size_t)hq * a.total_q + q0 + t : ((size_t)b * a.Hq + hq) * a.q_len + t;
+}
+
+template <int D, bool kVarlen>
 __device__ __forceinline__ void cursor_enter_row(Cursor &c, const DecodeArgs &a, int L) {
   constexpr int T = block_tokens(D);
   c.L = L;
   c.nb = (L + T - 1) / T;
+  if constexpr (kVarlen) {
+    c.q0 = c.q0_next;
+    c.qn = c.qn_next;
+    c.rtb = row_tiles(a, c.qn);
+    if (c.rtb == 0) c.nb = 0;  // a row without queries holds no units
+    if (c.b + 1 < a.B) row_queries<true>(a, c.b + 1, c.q0_next, c.qn_next);
+  } else {
+    c.q0 = c.b * a.q_len;
+    c.qn = a.q_len;
+  }
   c.L_next = c.b + 1 < a.B ? a.seqlens[c.b + 1] + a.len_add : 0;  // consumed a segment later
 }
 
 // The segment at the cursor (a contiguous block range of one unit); the
 // cursor moves past it, and past the fixed cost of the unit that follows.
-template <int D>
+template <int D, bool kVarlen>
 __device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
-  const int HR = a.Hkv * a.RT;
+  const int HR = a.Hkv * c.rtb;
   SegmentDesc s;
   const long long left = c.nb - c.blk, room = c.end - c.x;
   const int len = (int)(left < room ? left : room);
   s.b = c.b;
-  s.h = c.hr / a.RT;
-  s.rt = c.hr % a.RT;
+  s.h = c.hr / c.rtb;
+  s.rt = c.hr % c.rtb;
   s.blk_beg = c.blk;
   s.blk_end = c.blk + len;
   s.L = c.L;
@@ -113,7 +157,8 @@ __device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
     s.n_pieces = (c.nb + a.chunk_blocks - 1) / a.chunk_blocks;
   }
   s.last = 0;
-  s.pad[0] = s.pad[1] = 0;
+  s.q0 = c.q0;
+  s.qn = c.qn;
 
   c.x += len;
   c.blk += len;
@@ -123,10 +168,10 @@ __device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
       c.hr = 0;
       if (c.x + a.unit_cost < c.end && c.b + 1 < a.B) {
         ++c.b;
-        cursor_enter_row<D>(c, a, clamp_len(c.L_next, a.max_seqlen_k));
-        while (c.nb == 0 && c.b + 1 < a.B) {  // rows without keys hold no units
+        cursor_enter_row<D, kVarlen>(c, a, clamp_len(c.L_next, a.max_seqlen_k));
+        while (c.nb == 0 && c.b + 1 < a.B) {  // rows without keys (or queries) hold no units
           ++c.b;
-          cursor_enter_row<D>(c, a, clamp_len(a.seqlens[c.b] + a.len_add, a.max_seqlen_k));
+          cursor_enter_row<D, kVarlen>(c, a, clamp_len(a.seqlens[c.b] + a.len_add, a.max_seqlen_k));
         }
       } else {
         c.end = c.x;
@@ -141,9 +186,12 @@ __device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
 // to end (row-major over (b, KV head, row tile)) is cut into gridDim.x equal
 // ranges; the prefix sum over rows, and the lengths themselves, are kept in
 // the (still unused) ring by this warp alone, so the rows a range starts
-// and ends in are known without another read of global memory.  UNIFORM: block range [si * chunk, (si + 1) * chunk) of
-// unit blockIdx.x / splits.
-template <int D>
+// and ends in are known without another read of global memory.  With
+// per-row queries a row's scan width covers one KV head's row tiles (the
+// row's tile count is its width over a unit's), and the row's own query
+// offsets are read again where a range starts.  UNIFORM: block range
+// [si * chunk, (si + 1) * chunk) of unit blockIdx.x / splits.
+template <int D, bool kVarlen>
 __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cursor &tail, bool &has_tail) {
   constexpr int T = block_tokens(D);
   const int HR = a.Hkv * a.RT;
@@ -154,14 +202,18 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
   c.x = c.end = 0;
   c.per_cta = 1;
   c.L = c.nb = c.L_next = 0;
+  c.rtb = a.RT;
+  c.q0 = c.qn = c.q0_next = c.qn_next = 0;
   has_tail = false;
   tail = c;
   if (a.schedule == MXA_SCHED_UNIFORM) {
     const int u = blockIdx.x / a.splits, si = blockIdx.x % a.splits;
     c.b = u / HR;
     c.hr = u % HR;
+    row_queries<kVarlen>(a, c.b, c.q0, c.qn);
     c.L = clamp_len(a.seqlens[c.b] + a.len_add, a.max_seqlen_k);
     c.nb = (c.L + T - 1) / T;
+    if (kVarlen && c.hr % a.RT >= row_tiles(a, c.qn)) c.nb = 0;  // a tile past the row's queries
     const int beg = si * a.chunk_blocks, end = min(beg + a.chunk_blocks, c.nb);
     c.blk = beg;
     c.x = beg;
@@ -178,7 +230,12 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
     const int L = clamp_len(a.seqlens[i] + a.len_add, a.max_seqlen_k);
     lens[i] = L;
     const int nb = (L + T - 1) / T;
-    const int w = nb > 0 ? nb + V : 0;  // positions of one unit of row i
+    int w = nb > 0 ? nb + V : 0;  // positions of one unit of row i
+    if constexpr (kVarlen) {      // times the row's tiles: one KV head's units
+      int q0, qn;
+      row_queries<true>(a, i, q0, qn);
+      w *= row_tiles(a, qn);
+    }
     scan[i] = w;
     sum += w;
   }
@@ -196,7 +253,8 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
     scan[i] = run;  // inclusive prefix of unit positions per row
   }
   __syncwarp();
-  const long long NB = (long long)HR * total;
+  const long long HS = kVarlen ? a.Hkv : HR;  // a row spans HS times its scan width
+  const long long NB = HS * total;
   c.per_cta = NB == 0 ? 1 : (NB + gridDim.x - 1) / gridDim.x;
   const long long x0 = (long long)blockIdx.x * c.per_cta;
   c.b = 0;
@@ -205,15 +263,25 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
     int lo_b = 0, hi_b = a.B - 1;  // first row whose positions end past x0
     while (lo_b < hi_b) {
       const int mid = (lo_b + hi_b) >> 1;
-      if ((long long)HR * scan[mid] > x0) hi_b = mid; else lo_b = mid + 1;
+      if (HS * scan[mid] > x0) hi_b = mid; else lo_b = mid + 1;
     }
     const long long pre = lo_b > 0 ? scan[lo_b - 1] : 0;
     const long long w = scan[lo_b] - pre;  // > 0: the row holds position x0
-    const long long off = x0 - (long long)HR * pre;
-    const long long pos = off % w;
+    const long long off = x0 - HS * pre;
+    // positions of one unit of the row (from the scan, or its length)
+    const long long uw = kVarlen ? (long long)((lens[lo_b] + T - 1) / T + V) : w;
+    const long long pos = off % uw;
     c.b = lo_b;
-    c.hr = (int)(off / w);
-    c.nb = (int)(w - V);  // from the scan: the length itself is first needed later
+    c.hr = (int)(off / uw);
+    c.nb = (int)(uw - V);
+    if constexpr (kVarlen) {
+      c.rtb = (int)(w / uw);
+      row_queries<true>(a, lo_b, c.q0, c.qn);
+      if (lo_b + 1 < a.B) row_queries<true>(a, lo_b + 1, c.q0_next, c.qn_next);
+    } else {
+      c.q0 = lo_b * a.q_len;
+      c.qn = a.q_len;
+    }
     c.blk = pos > V ? (int)(pos - V) : 0;
     c.x = x0 - pos + V + c.blk;
     c.end = x1;
@@ -228,18 +296,19 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
     int lb = lo_b, hb = a.B - 1;
     while (lb < hb) {
       const int mid = (lb + hb) >> 1;
-      if ((long long)HR * scan[mid] > xl) hb = mid; else lb = mid + 1;
+      if (HS * scan[mid] > xl) hb = mid; else lb = mid + 1;
     }
     const long long pre_l = lb > 0 ? scan[lb - 1] : 0;
     const long long w_l = scan[lb] - pre_l;
-    const long long off_l = xl - (long long)HR * pre_l;
-    const long long pos_l = off_l % w_l;
+    const long long off_l = xl - HS * pre_l;
+    const long long uw_l = kVarlen ? (long long)((lens[lb] + T - 1) / T + V) : w_l;
+    const long long pos_l = off_l % uw_l;
     if (pos_l >= V) {  // xl falls on a KV block of that unit
-      const int nb_l = (int)(w_l - V), blk_l = (int)(pos_l - V);
+      const int nb_l = (int)(uw_l - V), blk_l = (int)(pos_l - V);
       const long long x_t = xl - blk_l;  // position of that unit's first block
       if (blk_l + 1 < nb_l && x_t - V > x0) {
         tail.b = lb;
-        tail.hr = (int)(off_l / w_l);
+        tail.hr = (int)(off_l / uw_l);
         tail.blk = 0;
         tail.x = x_t;
         tail.end = x1;
@@ -247,6 +316,13 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
         tail.nb = nb_l;
         tail.L = lens[lb];
         tail.L_next = 0;
+        if constexpr (kVarlen) {
+          tail.rtb = (int)(w_l / uw_l);
+          row_queries<true>(a, lb, tail.q0, tail.qn);
+        } else {
+          tail.q0 = lb * a.q_len;
+          tail.qn = a.q_len;
+        }
         has_tail = true;
         c.end = x_t - V;  // the main walk stops where that unit begins
       }
@@ -267,9 +343,10 @@ __device__ __forceinline__ int bt_entry(const DecodeArgs &a, int b, int p, int n
   return p < npages ? a.block_table[(size_t)b * a.mpps + p] : 0;
 }
 
-// kAppend: the call appends new tokens to the cache (len_add > 0); the plain
-// decode instance carries none of that code.
-template <int D, bool kBf16, bool kAppend>
+// kAppend: the call appends new tokens to the cache (len_add > 0); kVarlen:
+// every row has its own query count (offsets cu_q).  The plain decode
+// instance carries none of that code.
+template <int D, bool kBf16, bool kAppend, bool kVarlen>
 __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *smem, int lane) {
   constexpr int T = block_tokens(D);
   constexpr int CH = D / 64;
@@ -295,35 +372,36 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
   grid_dependency_wait();
   Cursor tail;
   bool has_tail;
-  Cursor cur = cursor_start<D>(a, smem, lane, tail, has_tail);
+  Cursor cur = cursor_start<D, kVarlen>(a, smem, lane, tail, has_tail);
   auto more = [&]() { return has_tail || (cur.x < cur.end && cur.nb > 0); };
   // Publish the units of this CTA that are split across CTAs (at most the
   // first unit of its range and the tail unit): the epilogue warp tags their
   // arrival counters with this launch's epoch before any piece is counted.
   if (lane == 0) {
-    const int HR = a.Hkv * a.RT;
+    // unit id (b, KV head, row tile) of a cursor's unit, over the plan's RT tiles per row
+    auto unit_of = [&](const Cursor &k) { return (k.b * a.Hkv + k.hr / k.rtb) * a.RT + k.hr % k.rtb; };
     int u_first = -1;
     if (cur.x < cur.end && cur.nb > 0) {
       const bool split = a.schedule == MXA_SCHED_BALANCED ? (cur.blk > 0 || cur.x - cur.blk + cur.nb > cur.end)
                                                           : cur.nb > a.chunk_blocks;
-      if (split) u_first = cur.b * HR + cur.hr;
+      if (split) u_first = unit_of(cur);
     }
     int *init_units = reinterpret_cast<int *>(smem + smem_bar_off(D) + kInitUnitsOff);
     init_units[0] = u_first;
-    init_units[1] = has_tail ? tail.b * HR + tail.hr : -1;
+    init_units[1] = has_tail ? unit_of(tail) : -1;
     mbar_arrive(bar_addr(smem, D, B_INIT));
   }
   auto take = [&]() {
     if (has_tail) {
       has_tail = false;
-      return cursor_take<D>(tail, a);
+      return cursor_take<D, kVarlen>(tail, a);
     }
-    return cursor_take<D>(cur, a);
+    return cursor_take<D, kVarlen>(cur, a);
   };
 
   // Publish a segment to the math warps: its descriptor and its Q tile.
   auto issue_q = [&](const SegmentDesc &s) {
-    const int rows = min(kRowsPerTile, a.M - s.rt * kRowsPerTile);
+    const int rows = tile_rows(a, s.qn, s.rt);
     if (lane == 0) {
       *desc = s;
       mbar_arrive_expect_tx(qfull, (uint32_t)rows * D * 2);
@@ -332,7 +410,7 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
     if (lane < rows) {
       const int m = s.rt * kRowsPerTile + lane;
       const int t = m / a.G, g = m % a.G;
-      const uint16_t *src = q + ((size_t)(s.b * a.q_len + t) * a.Hq + (size_t)s.h * a.G + g) * D;
+      const uint16_t *src = q + ((size_t)(s.q0 + t) * a.Hq + (size_t)s.h * a.G + g) * D;
       bulk_load(qtile + (uint32_t)lane * q_row_pitch(D), src, D * 2, qfull);
     }
   };
@@ -360,7 +438,12 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
         const int idx = p / ps - w.base;
         const int va = __shfl_sync(0xffffffffu, w.wa, idx & 31);
         const int vb = __shfl_sync(0xffffffffu, w.wb, idx & 31);
-        token = (long long)(idx < 32 ? va : vb) * ps + p % ps;
+        const int page = idx < 32 ? va : vb;  // the same in every lane
+        if (page < 0 || page >= a.num_pages) {  // not a page of the pool: skip the token, report it
+          if (lane == 0) atomicOr(&g_mxa_err, kErrBadPage);
+          continue;
+        }
+        token = (long long)page * ps + p % ps;
       }
       if (lane < 2 * CW) {
         const bool is_v = lane >= CW;
@@ -375,6 +458,7 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
   int it = 0;     // KV stages issued
   int seg_k = 0;  // segments published
   bool ok = true;
+  bool bad_page = false;  // a block-table entry outside [0, num_pages) was met
   if (more()) {
     SegmentDesc seg = take();
     seg.last = more() ? 0 : 1;
@@ -435,6 +519,10 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
             const int va = __shfl_sync(0xffffffffu, win.wa, src);
             const int vb = __shfl_sync(0xffffffffu, win.wb, src);
             page = idx < 32 ? va : vb;
+            if (page < 0 || page >= a.num_pages) {  // not a page of the pool: read as zeros, reported
+              bad_page |= op < n_ops;
+              page = -1;  // rows [-page_size, 0): outside the map, so the box is filled with zeros
+            }
           }
           if (op < n_ops) {
             const int row = a.contiguous ? seg.b * ps + tok : page * ps + tok % ps;
@@ -483,6 +571,7 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
     }
   }
 
+  if (__any_sync(0xffffffffu, bad_page) && lane == 0) atomicOr(&g_mxa_err, kErrBadPage);
   if (ok && warp_wait_bounded(qempty, (seg_k & 1) ^ 1, &g_mxa_err, kErrWaitQ, lane)) {
     if (lane == 0) {  // end-of-work marker for the math warps
       SegmentDesc d{};
@@ -546,6 +635,7 @@ __device__ void math_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lan
     if (!warp_wait_bounded(qfull, seg_k & 1, &g_mxa_err, kErrWaitQ, lane)) return;
     const int b = desc[0], h = desc[1], rt = desc[2], blk_beg = desc[3], blk_end = desc[4];
     const int L = desc[5], kind = desc[6], c_first = desc[7], n_pieces = desc[8], last = desc[9];
+    const int q0 = desc[10], qn = desc[11];
     const int j = seg_k % kJobs, jk = seg_k / kJobs;
     if (kind < 0) {  // end of work: pass the marker on to the epilogue warp
       if (!warp_wait_bounded(bar_addr(smem, D, B_JOBEMPTY(j)), (jk & 1) ^ 1, &g_mxa_err, kErrWaitQ, lane))
@@ -555,7 +645,7 @@ __device__ void math_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lan
       if (lane == 0) mbar_arrive(bar_addr(smem, D, B_JOBFULL(j)));
       return;
     }
-    const int rows = min(kRowsPerTile, a.M - rt * kRowsPerTile);
+    const int rows = tile_rows(a, qn, rt);
 
     // Q tile -> A fragments, resident in registers for the whole segment
     uint32_t qa[KS][4];
@@ -576,9 +666,9 @@ __device__ void math_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lan
     int lim0 = L, lim1 = L, tile_lim = L;
     if (a.causal) {
       const int m0 = rt * kRowsPerTile + r, m1 = m0 + 8;
-      if (r < rows) lim0 = min(L, L - a.q_len + m0 / a.G + 1);
-      if (r + 8 < rows) lim1 = min(L, L - a.q_len + m1 / a.G + 1);
-      tile_lim = min(L, L - a.q_len + (rt * kRowsPerTile) / a.G + 1);
+      if (r < rows) lim0 = min(L, L - qn + m0 / a.G + 1);
+      if (r + 8 < rows) lim1 = min(L, L - qn + m1 / a.G + 1);
+      tile_lim = min(L, L - qn + (rt * kRowsPerTile) / a.G + 1);
     }
 
     float m_0 = NEG_INF, m_1 = NEG_INF, l_0 = 0.f, l_1 = 0.f;
@@ -743,7 +833,8 @@ __device__ void math_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lan
       sd.b = b; sd.h = h; sd.rt = rt; sd.blk_beg = blk_beg; sd.blk_end = blk_end; sd.L = L;
       sd.kind = kind; sd.c_first = c_first; sd.n_pieces = n_pieces;
       sd.last = last;
-      sd.pad[0] = sd.pad[1] = 0;
+      sd.q0 = q0;
+      sd.qn = qn;
       jobs[j].seg = sd;
       jobs[j].stage = s_last;
     }
@@ -756,18 +847,6 @@ __device__ void math_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lan
 // ---------------------------------------------------------------------------
 // Epilogue warp
 // ---------------------------------------------------------------------------
-
-// D / 32 consecutive output values of one row -> out[b, t, hq, col..]
-template <int D, bool kBf16>
-__device__ __forceinline__ void store_out_vec(const DecodeArgs &a, int b, int t, int hq, int col,
-                                              const float *v) {
-  uint16_t *dst = reinterpret_cast<uint16_t *>(a.out) + ((size_t)(b * a.q_len + t) * a.Hq + hq) * D + col;
-  if constexpr (D / 32 == 4) {
-    *reinterpret_cast<uint2 *>(dst) = make_uint2(pack2<kBf16>(v[0], v[1]), pack2<kBf16>(v[2], v[3]));
-  } else {
-    *reinterpret_cast<uint32_t *>(dst) = pack2<kBf16>(v[0], v[1]);
-  }
-}
 
 // D / 32 consecutive values of packed row `rr`, rounded to the output type,
 // into the staging rows at shared address `stage` (row pitch D * 2 bytes).
@@ -782,37 +861,43 @@ __device__ __forceinline__ void stage_out_vec(uint8_t *smem, uint32_t stage, int
   }
 }
 
-// Bulk stores of `rows` staged output rows of a unit: the rows of one query
-// position t are the consecutive heads h * G + g and so one contiguous run
-// of out[b, t, :, :].  Issued by the calling lane.
+// Bulk stores of `rows` staged output rows of a unit whose row's first
+// packed query token is q0: the rows of one query position t are the
+// consecutive heads h * G + g and so one contiguous run of
+// out[q0 + t, :, :].  Issued by the calling lane.
 template <int D>
-__device__ __forceinline__ void store_out_rows(const DecodeArgs &a, int b, int h, int rt, int rows,
+__device__ __forceinline__ void store_out_rows(const DecodeArgs &a, int q0, int h, int rt, int rows,
                                                uint32_t stage) {
   int r = 0;
   while (r < rows) {
     const int m = rt * kRowsPerTile + r, t = m / a.G, g = m % a.G;
     const int r_end = min(rows, (t + 1) * a.G - rt * kRowsPerTile);
-    uint16_t *dst = reinterpret_cast<uint16_t *>(a.out) + ((size_t)(b * a.q_len + t) * a.Hq + (size_t)h * a.G + g) * D;
+    uint16_t *dst = reinterpret_cast<uint16_t *>(a.out) + ((size_t)(q0 + t) * a.Hq + (size_t)h * a.G + g) * D;
     bulk_store(dst, stage + (uint32_t)(r * D * 2), (uint32_t)((r_end - r) * D * 2));
     r = r_end;
   }
 }
 
 // Output of a unit whose row sees no key at all (L_b = 0): O = 0, LSE = -inf.
+// A tile past the row's queries (per-row query counts) has no output.
 template <int D>
 __device__ void write_empty_unit(const DecodeArgs &a, int unit, int lane) {
   const int rt = unit % a.RT, hr = unit / a.RT, h = hr % a.Hkv, b = hr / a.Hkv;
-  const int rows = min(kRowsPerTile, a.M - rt * kRowsPerTile);
+  int q0, qn;
+  if (a.cu_q != nullptr) row_queries<true>(a, b, q0, qn);
+  else row_queries<false>(a, b, q0, qn);
+  if (rt >= row_tiles(a, qn)) return;  // the same for every lane
+  const int rows = tile_rows(a, qn, rt);
   uint16_t *out = reinterpret_cast<uint16_t *>(a.out);
   for (int i = lane; i < rows * D; i += 32) {
     const int rr = i / D, d = i % D;
     const int m = rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G;
-    out[((size_t)(b * a.q_len + t) * a.Hq + (size_t)h * a.G + g) * D + d] = 0;  // +0 in fp16 and bf16
+    out[((size_t)(q0 + t) * a.Hq + (size_t)h * a.G + g) * D + d] = 0;  // +0 in fp16 and bf16
   }
   if (a.lse != nullptr) {
     for (int rr = lane; rr < rows; rr += 32) {
       const int m = rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G;
-      a.lse[((size_t)b * a.Hq + (size_t)h * a.G + g) * a.q_len + t] = -INFINITY;
+      a.lse[lse_index(a, b, q0, h * a.G + g, t)] = -INFINITY;
     }
   }
   __syncwarp();
@@ -917,7 +1002,7 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
   const float lse2 = sm > 0.f ? mx + log2f(sm) : -INFINITY;  // this row's LSE, base 2
   if (r1 < rows && j1 == 0 && a.lse != nullptr) {
     const int mrow = sg.rt * kRowsPerTile + r1, t = mrow / a.G, g = mrow % a.G;
-    a.lse[((size_t)sg.b * a.Hq + (size_t)sg.h * a.G + g) * a.q_len + t] = lse2 * kLn2;
+    a.lse[lse_index(a, sg.b, sg.q0, sg.h * a.G + g, t)] = lse2 * kLn2;
   }
   // With every LSE landed, the lanes that read a piece's LSE turn it into
   // its weight exp(lse_i - LSE) in place, once for all lanes.
@@ -976,7 +1061,7 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
   fence_proxy_async_smem();  // staged rows are read by the bulk stores
   __syncwarp();
   if (lane == 0) {
-    store_out_rows<D>(a, sg.b, sg.h, sg.rt, rows, ostage);
+    store_out_rows<D>(a, sg.q0, sg.h, sg.rt, rows, ostage);
     bulk_commit();
     a.counters[unit] = 0ull;  // every piece has arrived; leave it clean
   }
@@ -1063,7 +1148,7 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
     // the staging rows are free once earlier bulk stores have read them
     if (lane == 0) bulk_wait_read_all();
     __syncwarp();
-    const int rows = min(kRowsPerTile, a.M - sg.rt * kRowsPerTile);
+    const int rows = tile_rows(a, sg.qn, sg.rt);
     const int unit = (sg.b * a.Hkv + sg.h) * a.RT + sg.rt;
     const int slot = sg.kind - 1;  // partial slot (kind 1 -> head slot 0, kind 2 -> tail slot 1)
     // A piece of a split unit reads the unit's count now (acquire); the read
@@ -1177,7 +1262,7 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
     if (lane < rows) {
       if (sg.kind == 0) {
         const int m = sg.rt * kRowsPerTile + lane, t = m / a.G, g = m % a.G, hq = sg.h * a.G + g;
-        if (a.lse != nullptr) a.lse[((size_t)sg.b * a.Hq + hq) * a.q_len + t] = my_lse;
+        if (a.lse != nullptr) a.lse[lse_index(a, sg.b, sg.q0, hq, t)] = my_lse;
       } else if (merge_now) {  // at this piece's index among the landed LSEs
         reinterpret_cast<float *>(smem + (land + land_rows - smem_addr(smem)))[own * kRowsPerTile + lane] = my_lse;
       } else {  // after the 16 staged rows; stored with them
@@ -1194,7 +1279,7 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
       mbar_arrive(bar_addr(smem, D, B_JOBEMPTY(j)));
       if (!hold) mbar_arrive_cnt(bar_addr(smem, D, B_EMPTY(stage)), kMathWarps);
       if (sg.kind == 0) {
-        store_out_rows<D>(a, sg.b, sg.h, sg.rt, rows, ostage);
+        store_out_rows<D>(a, sg.q0, sg.h, sg.rt, rows, ostage);
       } else if (!merge_now) {
         const size_t ps = (size_t)blockIdx.x * 2 + slot;
         bulk_store(a.o_part + ps * kRowsPerTile * D, ostage, (uint32_t)(rows * D * 4));
@@ -1239,7 +1324,7 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
 // ---------------------------------------------------------------------------
 // The split kernel
 // ---------------------------------------------------------------------------
-template <int D, bool kBf16, bool kAppend>
+template <int D, bool kBf16, bool kAppend, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 2)
     mxa_split_kernel(const __grid_constant__ TmapPair tm, const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -1270,7 +1355,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   // warps).  The math warps touch shared memory only.
   grid_launch_dependents();
   if (warp == kProducerWarp) {
-    producer_warp<D, kBf16, kAppend>(tm, a, smem, lane);
+    producer_warp<D, kBf16, kAppend, kVarlen>(tm, a, smem, lane);
   } else if (warp == kEpilogueWarp) {
     epilogue_warp<D, kBf16>(a, smem, lane);
   } else {
@@ -1400,13 +1485,13 @@ bool kv_maps(TmapPair *tm, const void *k, const void *v, int D, int Hkv, long lo
   return true;
 }
 
-template <int D, bool kBf16, bool kAppend>
+template <int D, bool kBf16, bool kAppend, bool kVarlen>
 cudaError_t prepare_split_kernel(int device) {
   static std::mutex mu;
   static bool done[kMaxDevices] = {};
   std::lock_guard<std::mutex> lock(mu);
   if (device >= 0 && device < kMaxDevices && done[device]) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(mxa_split_kernel<D, kBf16, kAppend>,
+  cudaError_t e = cudaFuncSetAttribute(mxa_split_kernel<D, kBf16, kAppend, kVarlen>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_total(D));
   if (e == cudaSuccess && device >= 0 && device < kMaxDevices) done[device] = true;
   return e;
@@ -1427,13 +1512,17 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
   const mxa_plan_t &plan = L.plan;
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return MXA_ERR_CUDA;
-  const bool append = L.len_add > 0;
-  if ((append ? prepare_split_kernel<D, kBf16, true>(device) : prepare_split_kernel<D, kBf16, false>(device)) !=
-      cudaSuccess)
-    return MXA_ERR_CUDA;
+  const bool append = L.len_add > 0, varlen = L.cu_q != nullptr;
+  if (append && varlen) return MXA_ERR_UNSUPPORTED;
+  const cudaError_t pe = append   ? prepare_split_kernel<D, kBf16, true, false>(device)
+                         : varlen ? prepare_split_kernel<D, kBf16, false, true>(device)
+                                  : prepare_split_kernel<D, kBf16, false, false>(device);
+  if (pe != cudaSuccess) return MXA_ERR_CUDA;
 
   DecodeArgs a{};
   a.q = L.q;
+  a.cu_q = L.cu_q;
+  a.total_q = varlen ? L.total_q : p.B * p.q_len;
   a.block_table = L.block_table;
   a.seqlens = L.seqlens;
   a.out = L.out;
@@ -1447,6 +1536,7 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
   a.RT = (a.M + kRowsPerTile - 1) / kRowsPerTile;
   a.contiguous = L.block_table == nullptr;
   a.page_size = p.page_size;
+  a.num_pages = p.num_pages;
   a.mpps = p.max_pages_per_seq;
   a.max_seqlen_k = p.max_seqlen_k;
   a.box_tokens = a.contiguous ? T : (p.page_size % T == 0 ? T : p.page_size);
@@ -1486,8 +1576,9 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = append ? cudaLaunchKernelEx(&cfg, mxa_split_kernel<D, kBf16, true>, tm, a)
-                               : cudaLaunchKernelEx(&cfg, mxa_split_kernel<D, kBf16, false>, tm, a);
+  const cudaError_t e = append   ? cudaLaunchKernelEx(&cfg, mxa_split_kernel<D, kBf16, true, false>, tm, a)
+                        : varlen ? cudaLaunchKernelEx(&cfg, mxa_split_kernel<D, kBf16, false, true>, tm, a)
+                                 : cudaLaunchKernelEx(&cfg, mxa_split_kernel<D, kBf16, false, false>, tm, a);
   if (e != cudaSuccess) return MXA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? MXA_OK : MXA_ERR_CUDA;
 }

@@ -18,16 +18,19 @@ struct alignas(64) TmapPair {
 };
 
 struct DecodeArgs {
-  const void *q;               // [B, q_len, Hq, D]
+  const void *q;               // [B, q_len, Hq, D], or [total_q, Hq, D] with cu_q
+  const int32_t *cu_q;         // [B + 1] offsets of each row's queries (varlen), or null
   const int32_t *block_table;  // [B, mpps] (unused when contiguous)
   const int32_t *seqlens;      // [B]
-  void *out;                   // [B, q_len, Hq, D]
-  float *lse;                  // [B, Hq, q_len] or null
+  void *out;                   // [B, q_len, Hq, D], or [total_q, Hq, D] with cu_q
+  float *lse;                  // [B, Hq, q_len], or [Hq, total_q] with cu_q; or null
   unsigned long long *counters;  // [units]: epoch-tagged arrivals of split units
   float *lse_part;             // [grid][2][16]
   float *o_part;               // [grid][2][16][D]
-  int B, q_len, Hq, Hkv, G, M, RT;
+  int B, q_len, Hq, Hkv, G, M, RT;  // varlen: q_len bounds every row's query count
+  int total_q;                 // varlen: packed query tokens
   int page_size;               // slots per page (row capacity when contiguous)
+  int num_pages;               // pages in the pool (paged)
   int mpps;                    // block-table row stride
   int contiguous;
   int max_seqlen_k;
@@ -60,6 +63,8 @@ struct DecodeLaunch {
   int causal;
   int len_add;  // q_len when the call appends the new tokens first, else 0
   const void *k_new, *v_new;  // [B, q_len, Hkv, D] when len_add > 0
+  const int32_t *cu_q;        // varlen: [B + 1] query offsets (null: q_len queries per row)
+  int total_q;                // varlen: packed query tokens
 };
 
 // Launch the split kernel (split units are merged inside it).

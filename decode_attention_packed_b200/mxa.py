@@ -30,7 +30,7 @@ MXA_SCHED_UNIFORM, MXA_SCHED_BALANCED = 0, 1
 EXPORTED = ("mxa_status_string", "mxa_should_pack_gqa", "mxa_num_splits_heuristic", "mxa_plan",
             "mxa_plan_balanced",
             "mxa_decode_fwd", "mxa_decode_fwd_with_plan", "mxa_combine", "mxa_device_error",
-            "mxa_decode_fwd_noalloc", "mxa_decode_fwd_append")
+            "mxa_decode_fwd_noalloc", "mxa_decode_fwd_append", "mxa_decode_fwd_varlen")
 
 
 class mxa_decode_params_t(ctypes.Structure):
@@ -74,6 +74,10 @@ _lib.mxa_decode_fwd_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, ctypes.POINTE
                                        ctypes.c_float, _I, ctypes.POINTER(mxa_plan_t), _P, ctypes.c_size_t,
                                        _P, _P, _P]
 _lib.mxa_decode_fwd_append.restype = _I
+_lib.mxa_decode_fwd_varlen.argtypes = [_P, _P, _I, _P, _P, _P, _P, ctypes.POINTER(mxa_decode_params_t),
+                                       ctypes.c_float, _I, ctypes.POINTER(mxa_plan_t), _P, ctypes.c_size_t,
+                                       _P, _P, _P]
+_lib.mxa_decode_fwd_varlen.restype = _I
 _lib.mxa_decode_fwd_noalloc.argtypes = [_P, _P, _P, _P, _P, ctypes.POINTER(mxa_decode_params_t),
                                         ctypes.c_float, _I, _I, _P, _P, _P]
 _lib.mxa_decode_fwd_noalloc.restype = _I
@@ -163,6 +167,18 @@ def mxa_decode_fwd_append(q, k_cache, v_cache, k_new, v_new, block_table, cache_
                                       _ptr(block_table), _ptr(cache_seqlens), ctypes.byref(params),
                                       float(scale), int(causal), ctypes.byref(plan), _ptr(workspace), ws_bytes,
                                       _ptr(out), _ptr(lse), _stream(stream)), "mxa_decode_fwd_append")
+
+
+def mxa_decode_fwd_varlen(q, cu_seqlens_q, k_cache, v_cache, block_table, cache_seqlens, params, scale,
+                          causal, plan, workspace, out, lse, stream=None) -> None:
+    """Decode rows with their own query counts: q [total_q, Hq, D], row b's
+    queries at cu_seqlens_q[b] .. cu_seqlens_q[b + 1] - 1; params.q_len bounds
+    every count.  out [total_q, Hq, D], lse [Hq, total_q] (see mxa.h)."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.mxa_decode_fwd_varlen(_ptr(q), _ptr(cu_seqlens_q), int(q.shape[0]), _ptr(k_cache),
+                                      _ptr(v_cache), _ptr(block_table), _ptr(cache_seqlens), ctypes.byref(params),
+                                      float(scale), int(causal), ctypes.byref(plan), _ptr(workspace), ws_bytes,
+                                      _ptr(out), _ptr(lse), _stream(stream)), "mxa_decode_fwd_varlen")
 
 
 def mxa_decode_fwd_noalloc(q, k_cache, v_cache, block_table, cache_seqlens, params, scale, causal,
@@ -261,4 +277,32 @@ def decode(q, k_cache, v_cache, block_table, cache_seqlens, *, scale=None, causa
     else:
         mxa_decode_fwd_append(q, k_cache, v_cache, k_new, v_new, block_table, cache_seqlens, prepared.params,
                               scale, causal, prepared.plan, prepared.workspace, out, lse, stream)
+    return out, lse
+
+
+def decode_varlen(q, cu_seqlens_q, k_cache, v_cache, block_table, cache_seqlens, *, max_seqlen_q,
+                  scale=None, causal=False, num_splits=0, max_seqlen_k=None, out=None, lse=None,
+                  prepared: Optional[Prepared] = None, return_lse=True, stream=None):
+    """out [total_q, Hq, D] (and lse [Hq, total_q] fp32) for rows with their
+    own query counts: q [total_q, Hq, D], cu_seqlens_q [B + 1] int32 on the
+    device, max_seqlen_q >= every row's count (it sizes the plan)."""
+    total_q, Hq, D = q.shape
+    B = cu_seqlens_q.shape[0] - 1
+    if scale is None:
+        scale = D ** -0.5
+    if prepared is None:
+        # planned as B rows of max_seqlen_q queries (a shape-only tensor)
+        shape = torch.empty((B, int(max_seqlen_q), Hq, D), dtype=q.dtype, device="meta")
+        params = params_for(shape, k_cache, block_table, max_seqlen_k)
+        plan = mxa_plan(params, num_splits)
+        ws = None
+        if plan.workspace_bytes:
+            ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=q.device)
+        prepared = Prepared(params, plan, ws)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    mxa_decode_fwd_varlen(q, cu_seqlens_q, k_cache, v_cache, block_table, cache_seqlens, prepared.params,
+                          scale, causal, prepared.plan, prepared.workspace, out, lse, stream)
     return out, lse

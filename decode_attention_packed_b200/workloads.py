@@ -76,7 +76,15 @@ WORKLOADS = [
              page_size=16, causal=False, lengths="loguniform:1:16384", k_scale=3.0, seed=1004),
 ]
 
-BY_NAME = {w.name: w for w in WORKLOADS}
+# Other readings of the workloads above, benchmarked for context only: the
+# speculative step with every row at 8192 keys (the spec/MTP lengths read as
+# "all rows 8192" instead of the cycle through the non-power-of-two lengths).
+CONTEXT_WORKLOADS = [
+    Workload("spec_mtp_small_q_all8192", B=16, q_len=4, Hq=32, Hkv=8, D=128, dtype="bf16",
+             page_size=64, causal=True, lengths="const:8192", seed=1012),
+]
+
+BY_NAME = {w.name: w for w in WORKLOADS + CONTEXT_WORKLOADS}
 
 
 def workload(name_or_index) -> Workload:
@@ -176,6 +184,18 @@ def make_inputs(w: Workload, seed: Optional[int] = None,
                   v_cache=_round(v, w.dtype), block_table=block_table,
                   cache_seqlens=torch.from_numpy(L.copy()), page_size=page,
                   max_seqlen_k=max_seqlen_k)
+
+
+def make_varlen_queries(q_lens, Hq: int, D: int, dtype: str, seed: int):
+    """Queries of rows with their own query counts, packed: q [total_q, Hq, D]
+    (N(0, 1) rounded to `dtype`) and the offsets cu [B + 1] int32 (0, then the
+    running totals of q_lens)."""
+    rng = np.random.default_rng(seed)
+    ql = np.asarray(q_lens, dtype=np.int64)
+    assert ql.ndim == 1 and (ql >= 0).all()
+    cu = np.concatenate([[0], np.cumsum(ql)]).astype(np.int32)
+    q = rng.standard_normal((int(cu[-1]), Hq, D), dtype=np.float32)
+    return _round(q, dtype), torch.from_numpy(cu)
 
 
 def small_variant(w: Workload, **changes) -> Workload:

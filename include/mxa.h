@@ -83,6 +83,9 @@ typedef enum { MXA_SCHED_UNIFORM = 0, MXA_SCHED_BALANCED = 1 } mxa_schedule_t;
  *                [B, page_size, Hkv, D]             dtype   (contiguous: block_table == NULL,
  *                                                            num_pages == B, page_size = row capacity)
  *   block_table  [B, max_pages_per_seq] int32: page id of logical page p of row b
+ *                (an id outside [0, num_pages) is never dereferenced: its keys
+ *                and values read as zeros, and mxa_device_error reports
+ *                MXA_ERR_INVALID_ARG)
  *   cache_seqlens[B] int32: number of valid keys L_b, 0 <= L_b <= max_seqlen_k
  *   out          [B, q_len, Hq, D]                 dtype
  *   lse          [B, Hq, q_len]                    float32, natural log
@@ -220,7 +223,9 @@ MXA_API mxa_status_t mxa_decode_fwd_with_plan(const void *q, const void *k_cache
  * Every query row then attends to the first L_b + q_len keys; with causal = 1
  * query t sees the first L_b + t + 1.  params->max_seqlen_k bounds L_b + q_len
  * (tokens that would land at or past it, or past the row's block-table
- * width, are not written).  The plan is that of mxa_plan for `params`.  One
+ * width, are not written; nor is a token whose page id lies outside
+ * [0, num_pages): mxa_device_error then reports MXA_ERR_INVALID_ARG).  The
+ * plan is that of mxa_plan for `params`.  One
  * kernel runs on `stream`: the CTA that streams the block holding an
  * appended token writes the token into the cache (for its KV head) and then
  * loads the block, so each token is written before it is read.
@@ -230,6 +235,34 @@ MXA_API mxa_status_t mxa_decode_fwd_append(const void *q, void *k_cache, void *v
                                            const int32_t *cache_seqlens, const mxa_decode_params_t *params,
                                            float scale, int causal, const mxa_plan_t *plan, void *workspace,
                                            size_t workspace_bytes, void *out, float *lse, void *stream);
+
+/* Decode rows that each have their own number of queries: the packed
+ * (varlen) layout of flash_attn_varlen_func ("MXFlashAttn 1.4.0", its API
+ * list), with the cu_seqlens_q offsets defined in
+ * "MixedQuantSparseFlashMlaMetadata 算子解析" (参数说明).
+ *   q            : device [total_q, Hq, D] dtype; row b's queries are
+ *                  q[cu_seqlens_q[b] .. cu_seqlens_q[b + 1] - 1]
+ *   cu_seqlens_q : device [B + 1] int32, read only: 0 = cu[0] <= cu[1] <= ...
+ *                  <= cu[B] = total_q
+ *   total_q      : packed query tokens (>= 0)
+ *   params->q_len: the largest per-row query count (max_seqlen_q); it sizes
+ *                  the plan (mxa_plan with these params) and the workspace
+ *   out          : device [total_q, Hq, D] dtype (written in full)
+ *   lse          : device [Hq, total_q] float32, or NULL to skip
+ * Row b with q_b = cu[b+1] - cu[b] queries: non-causal, every query sees L_b
+ * keys; causal, query t sees the first L_b - q_b + t + 1 (its queries are
+ * the row's last q_b cache entries).  A row with q_b = 0 writes nothing.
+ * Offsets are read on the device and not checked there against these rules:
+ * out-of-range values are clamped into [0, total_q] and a row's count to
+ * params->q_len, so that no access leaves the buffers, but the result of
+ * such a call is unspecified.  Other arguments and errors as
+ * mxa_decode_fwd_with_plan; MXA_ERR_INVALID_ARG for a NULL or misaligned
+ * cu_seqlens_q or total_q < 0. */
+MXA_API mxa_status_t mxa_decode_fwd_varlen(const void *q, const int32_t *cu_seqlens_q, int total_q,
+                                   const void *k_cache, const void *v_cache, const int32_t *block_table,
+                                   const int32_t *cache_seqlens, const mxa_decode_params_t *params,
+                                   float scale, int causal, const mxa_plan_t *plan, void *workspace,
+                                   size_t workspace_bytes, void *out, float *lse, void *stream);
 
 /* Decode without any device allocation, for callers that cannot allocate.
  * (An addition of this library; the source pages have no counterpart.)
@@ -276,9 +309,12 @@ MXA_API mxa_status_t mxa_combine(const float *o_part, const float *lse_part, int
                          void *stream);
 
 /* Synchronise the current device and report whether any kernel of this
- * library recorded a device-side failure (a bounded wait that ran out) since
- * the last reset: MXA_OK or MXA_ERR_TIMEOUT (MXA_ERR_CUDA if the device or
- * the synchronisation itself failed).  reset != 0 clears the record. */
+ * library recorded a device-side failure since the last reset: MXA_OK;
+ * MXA_ERR_TIMEOUT if a bounded wait ran out; else MXA_ERR_INVALID_ARG if a
+ * block-table entry that a kernel used lay outside [0, num_pages) (its keys
+ * read as zeros; an appended token there was not written); MXA_ERR_CUDA if
+ * the device or the synchronisation itself failed.
+ * reset != 0 clears the record. */
 MXA_API mxa_status_t mxa_device_error(int reset);
 
 #ifdef __cplusplus

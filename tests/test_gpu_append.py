@@ -128,3 +128,28 @@ def test_tokens_past_the_bound_are_not_written():
                            page_size=16, dtype="bf16", scale=w.scale, causal=False)
     assert_out_close(out.cpu(), ro, "bf16")
     assert_lse_close(lse.cpu(), rl)
+
+
+@pytest.mark.parametrize("bad_page", [10**6, -5])
+def test_an_out_of_pool_page_id_is_reported_and_not_written(bad_page):
+    # row 0's new token falls in a page whose id is not a page of the pool:
+    # the token is skipped and reported; row 1's token is written as usual
+    w = Workload(name="append_badpage", B=2, q_len=1, Hq=8, Hkv=2, D=128, dtype="bf16", page_size=16,
+                 causal=False, lengths="list:40,20", seed=540)
+    inp = make_inputs(w)
+    d = "cuda"
+    L = torch.tensor([39, 19], dtype=torch.int32)
+    bt = inp.block_table.clone()
+    bt[0, 39 // 16] = bad_page
+    k_new = torch.full((2, 1, 2, 128), 1.5, dtype=torch.bfloat16)
+    v_new = torch.full((2, 1, 2, 128), -2.0, dtype=torch.bfloat16)
+    kc, vc = inp.k_cache.to(d), inp.v_cache.to(d)
+    assert mxa.mxa_device_error(True) == mxa.MXA_OK
+    mxa.decode(inp.q.to(d), kc, vc, bt.to(d), L.to(d), scale=w.scale, causal=False, max_seqlen_k=40,
+               k_new=k_new.to(d), v_new=v_new.to(d))
+    torch.cuda.synchronize()
+    assert mxa.mxa_device_error(True) == mxa.MXA_ERR_INVALID_ARG
+    kx, vx = oracle.append_kv(inp.k_cache, inp.v_cache, k_new[1:], v_new[1:], inp.block_table[1:], L[1:].numpy(),
+                              page_size=16)  # row 1 only
+    assert np.array_equal(kc.cpu().view(torch.int16).numpy().view(np.uint16), kx)
+    assert np.array_equal(vc.cpu().view(torch.int16).numpy().view(np.uint16), vx)

@@ -308,3 +308,30 @@ def test_decode_replays_in_a_cuda_graph():
     torch.cuda.synchronize()
     assert mxa.mxa_device_error(True) == mxa.MXA_OK
     check(inp, out.cpu(), lse.cpu(), ref)
+
+
+@pytest.mark.parametrize("bad_page", [10**6, -5])
+def test_a_page_id_outside_the_pool_reads_as_zeros_and_is_reported(bad_page):
+    # row 1 (70 keys, pages of 16) has its logical page 2 pointing outside the
+    # pool: the call must attend to zeros there (as if that page held zero
+    # keys and values), leave the other rows alone, and report the entry
+    w = Workload(name="badpage", B=3, q_len=1, Hq=8, Hkv=2, D=128, dtype="bf16", page_size=16, causal=False,
+                 lengths="list:40,70,33", seed=545)
+    inp = make_inputs(w)
+    bt_bad = inp.block_table.clone()
+    bt_bad[1, 2] = bad_page
+    d = "cuda"
+    assert mxa.mxa_device_error(True) == mxa.MXA_OK
+    out, lse = mxa.decode(inp.q.to(d), inp.k_cache.to(d), inp.v_cache.to(d), bt_bad.to(d),
+                          inp.cache_seqlens.to(d), scale=w.scale, causal=False, max_seqlen_k=inp.max_seqlen_k)
+    torch.cuda.synchronize()
+    assert mxa.mxa_device_error(True) == mxa.MXA_ERR_INVALID_ARG
+    # the oracle on a pool with one more page, all zeros, in that entry's place
+    zero = torch.zeros((1,) + tuple(inp.k_cache.shape[1:]), dtype=inp.k_cache.dtype)
+    k_ref, v_ref = torch.cat([inp.k_cache, zero]), torch.cat([inp.v_cache, zero])
+    bt_ref = inp.block_table.clone()
+    bt_ref[1, 2] = inp.k_cache.shape[0]
+    ro, rl = oracle.decode(inp.q, k_ref, v_ref, bt_ref, inp.cache_seqlens, Hkv=w.Hkv, page_size=16, dtype=w.dtype,
+                           scale=w.scale, causal=False)
+    assert_out_close(out.cpu(), ro, w.dtype)
+    assert_lse_close(lse.cpu(), rl)

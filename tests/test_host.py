@@ -236,6 +236,28 @@ def test_shapes_whose_position_sums_overflow_are_refused():
     assert e.value.code == mxa.MXA_ERR_UNSUPPORTED
 
 
+def test_varlen_refuses_bad_arguments_before_launch():
+    p = params()
+    plan = mxa.mxa_plan(p, 0, sm_count=148)
+    f = lambda x: None if x is None else ctypes.c_void_p(x * 4096)
+    call = lambda **kw: mxa._lib.mxa_decode_fwd_varlen(
+        f(kw.get("q", 1)), kw.get("cu", f(1)), kw.get("total_q", 8), f(1), f(1), f(1), f(1),
+        ctypes.byref(kw.get("p", p)), 0.125, 0, ctypes.byref(kw.get("plan", plan)), f(1), 1 << 30, f(1), None,
+        None)
+    assert call(cu=None) == MXA_ERR_INVALID_ARG
+    assert call(cu=ctypes.c_void_p(4096 + 2)) == MXA_ERR_INVALID_ARG  # offsets are int32
+    assert call(total_q=-1) == MXA_ERR_INVALID_ARG
+    assert call(q=None) == MXA_ERR_INVALID_ARG
+    assert call(total_q=0) == MXA_OK  # no query: nothing to write, nothing launched
+    # a balanced plan whose per-row sums fit 32 bits for one row tile per
+    # head, but not for the two tiles (q_len 2 x 16 heads) a varlen row may use
+    big = params(B=1000, q_len=2, Hq=16, Hkv=1, D=128, page_size=64, num_pages=16,
+                 max_pages_per_seq=1073700, max_seqlen_k=1073700 * 64)
+    bplan = mxa.mxa_plan_balanced(big, 296, sm_count=148)
+    bplan.unit_cost = 64
+    assert call(p=big, plan=bplan) == mxa.MXA_ERR_UNSUPPORTED
+
+
 def test_combine_refuses_bad_arguments():
     f = lambda x: None if x is None else ctypes.c_void_p(x * 4096)
     c = mxa._lib.mxa_combine
