@@ -1,14 +1,25 @@
 """Benchmark: paged GQA decode attention on B200 through libmxa.so.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mxa|reference]
-                    [--workload gqa_decode] [--num-splits S]
+                    [--workload NAME] [--num-splits S] [--append | --varlen]
+                    [--no-suite] [--no-clocks]
 
-One step = one decode call (one launch of the split kernel, which also merges
-units split across CTAs) over the whole workload:
-B = 32 rows, Hq = 32, Hkv = 8, head_dim 128, bf16, pages of 16 slots in a
-seeded random permutation, KV lengths uniform in [1, 4096].  Inputs are
-seeded synthetic data.  KV pools rotate over three copies (each larger than
-L2) so no timed call reads KV from L2 left by the previous one.
+One step = one decode call (one launch of the split kernel, which also
+merges units split across CTAs) over the whole headline workload.  The
+headline is ragged_varlen, the largest of the decode workloads: B = 128
+rows, Hq = 16, Hkv = 8, head_dim 64, fp16, pages of 16 slots in a seeded
+random permutation, KV lengths log-uniform in [1, 16384], keys scaled by 3.
+Inputs are seeded synthetic data.  KV pools rotate over three device copies
+(each larger than L2) so that no timed call reads KV left in L2 by the
+previous one.
+
+Before the headline, the same run measures the other workloads that the
+throughput target covers (gqa_decode, spec_mtp_small_q,
+long_context_split_kv) the same way, each in its own timed region of K
+calls after W warm-up calls, with its own roofline and CPU baseline, plus
+per-call percentiles and, for long_context_split_kv, a table over
+num_splits.  They are reported under "workloads"; --no-suite skips them,
+and --workload NAME makes NAME the headline (and skips them too).
 
 Prints one JSON line (rank 0).  `value` is KV-read throughput in GB/s
 summed over ranks; `us_per_call` and the roofline block give the per-call
@@ -31,28 +42,33 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from decode_attention_packed_b200.workloads import WORKLOADS, make_inputs, make_varlen_queries, workload  # noqa: E402
+from decode_attention_packed_b200.workloads import make_inputs, make_varlen_queries, workload  # noqa: E402
 
 METRIC = "decode-attn µs/call and KV-read GB/s as % of B200 HBM peak (1 GPU)"
 
-# DRAM bytes (read + written) per launch of the split kernel on the default
-# workload, from an ncu capture (profiles/mxa_split_kernel_gqa_decode.md),
-# keyed by a hash of the kernel sources it was taken on: once the kernel
-# changes the number no longer applies and the bench reports null.
-MEASURED_TRAFFIC = {"b7634f37e38a8462": 248863488}
-DEFAULT_WORKLOAD = "gqa_decode"
+# DRAM bytes (read + written) per launch of the split kernel, from one ncu
+# capture per workload, keyed by a hash of the kernel sources the capture
+# was taken on: once the kernel changes, the figures no longer apply and
+# the bench reports null.  The captures and their commands are summarised
+# under profiles/.
+MEASURED_TRAFFIC = {}
+HEADLINE = "ragged_varlen"
+SUITE = ("gqa_decode", "spec_mtp_small_q", "long_context_split_kv")
+SPLIT_SWEEP = (1, 2, 4, 8, 16)
 FALLBACK_HBM_GBS = 6650.0
 N_POOLS = 3
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="mxa", choices=["mxa", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", default=None,
+                    help=f"headline workload (default {HEADLINE}, with the suite of the other gated workloads)")
     ap.add_argument("--num-splits", type=int, default=None)
+    ap.add_argument("--no-suite", action="store_true", help="measure the headline workload only")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--append", action="store_true",
                     help="each step also appends the step's q_len new tokens per row to the cache "
@@ -60,7 +76,15 @@ def parse():
     ap.add_argument("--varlen", action="store_true",
                     help="rows have their own query counts, drawn (seeded) from 1..q_len, packed with "
                          "cu_seqlens_q (mxa_decode_fwd_varlen)")
-    return ap.parse_args()
+    args = ap.parse_args(argv)
+    if args.warmup < 0 or args.steps < 1:
+        ap.error("--steps must be at least 1 and --warmup at least 0")
+    if args.append and args.varlen:
+        ap.error("--append and --varlen do not combine")
+    args.suite = args.workload is None and not args.no_suite
+    if args.workload is None:
+        args.workload = HEADLINE
+    return args
 
 
 def measured_peak():
@@ -112,7 +136,7 @@ def algorithmic_bytes(inp) -> dict:
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """nvidia-smi samples of SM clock and throttle reasons while the GPU works."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -120,7 +144,6 @@ class ClockSampler:
 
     def __init__(self, gpu_index: int, enabled: bool):
         self.proc = None
-        self.gpu = gpu_index
         if enabled:
             try:
                 self.proc = subprocess.Popen(
@@ -200,7 +223,7 @@ def omp_threads() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(inp, budget_s=12.0):
+def cpu_baseline(inp, budget_s):
     """The oracle, as it stands, on the host cores: whole passes over the
     workload until about `budget_s` seconds of CPU work are done."""
     dt, kv = oracle_cpu(inp)
@@ -247,140 +270,206 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    args = parse()
-    world, rank, local = setup_dist(args)
-    if args.impl == "reference":
-        run_reference(args, world, rank)
-        return
+class Runner:
+    """Device-side plumbing of one rank: stream, barriers, max over ranks."""
 
-    from decode_attention_packed_b200 import mxa
+    def __init__(self, world, rank, local):
+        self.world, self.rank, self.local = world, rank, local
+        self.dev = torch.device("cuda", local)
+        self.stream = torch.cuda.current_stream(self.dev)
 
-    w = workload(args.workload)
-    inp = shard_inputs(w, rank)
-    if args.append and args.varlen:
-        raise SystemExit("--append and --varlen do not combine")
-    dev = torch.device("cuda", local)
-    stream = torch.cuda.current_stream(dev)
-    q = inp.q.to(dev)
-    bt = None if inp.block_table is None else inp.block_table.to(dev)
-    sl = inp.cache_seqlens.to(dev)
-    pools = [(inp.k_cache.to(dev), inp.v_cache.to(dev))]
-    for _ in range(N_POOLS - 1):
-        pools.append((pools[0][0].clone(), pools[0][1].clone()))
-    splits = w.num_splits if args.num_splits is None else args.num_splits
-    prep = mxa.prepare(q, pools[0][0], bt, max_seqlen_k=inp.max_seqlen_k, num_splits=splits)
-    cu = hcu = None
-    if args.varlen:  # the plan above is for q_len queries per row, which bounds every row's count
-        q_lens = np.random.default_rng(w.seed + 77).integers(1, w.q_len + 1, size=w.B)
-        hqv, hcu = make_varlen_queries(q_lens, w.Hq, w.D, w.dtype, w.seed + 78)
-        q, cu = hqv.to(dev), hcu.to(dev)
-        hcu = hcu.pin_memory()
-    out = torch.empty_like(q)
-    lse = (torch.empty((w.Hq, q.shape[0]), dtype=torch.float32, device=dev) if args.varlen
-           else torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=dev))
-    nbytes = algorithmic_bytes(inp)
-    if args.append:  # the new tokens are read and written once more
-        nbytes["total"] += 2 * 2 * w.B * w.q_len * w.Hkv * w.D * inp.q.element_size()
-    launches_per_call = 1  # the split kernel merges split units itself
-
-    if args.append:
-        # the rows' last q_len keys arrive as this step's new tokens: the call
-        # writes them (the same values each step) and attends to all keys
-        sl_before = (sl - w.q_len).clamp(min=0)
-        k_new = torch.randn((w.B, w.q_len, w.Hkv, w.D), device=dev).to(q.dtype)
-        v_new = torch.randn_like(k_new)
-
-    def run(i, q, cu, bt, sl, out, lse):
-        k, v = pools[i % N_POOLS]
-        if args.append:
-            mxa.mxa_decode_fwd_append(q, k, v, k_new, v_new, bt, sl, prep.params, w.scale, w.causal,
-                                      prep.plan, prep.workspace, out, lse, stream)
-        elif args.varlen:
-            mxa.mxa_decode_fwd_varlen(q, cu, k, v, bt, sl, prep.params, w.scale, w.causal, prep.plan,
-                                      prep.workspace, out, lse, stream)
-        else:
-            mxa.mxa_decode_fwd_with_plan(q, k, v, bt, sl, prep.params, w.scale, w.causal, prep.plan,
-                                         prep.workspace, out, lse, stream)
-
-    def call(i):
-        run(i, q, cu, bt, sl_before if args.append else sl, out, lse)
-
-    def barrier():
-        if world > 1:
+    def barrier(self):
+        if self.world > 1:
             import torch.distributed as dist
-            dist.barrier(device_ids=[local])
-        torch.cuda.synchronize(dev)
+            dist.barrier(device_ids=[self.local])
+        torch.cuda.synchronize(self.dev)
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
+    def max_over_ranks(self, x: float) -> float:
+        if self.world == 1:
             return x
         import torch.distributed as dist
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        t = torch.tensor([x], dtype=torch.float64, device=self.dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    # ---- device-timed region: inputs resident in HBM ----
-    for i in range(args.warmup):
-        call(i)
-    barrier()
-    clocks = ClockSampler(local, enabled=not args.no_clocks)
-    time.sleep(0.25 if not args.no_clocks else 0)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    e0.record(stream)
-    for i in range(args.steps):
-        call(i)
-    e1.record(stream)
-    barrier()
-    clk = clocks.stop()
-    dev_s = max_over_ranks(e0.elapsed_time(e1) / 1e3)
-    assert mxa.mxa_device_error(True) == mxa.MXA_OK, "device-side wait ran out during the bench"
+    def timed(self, call, warmup, steps) -> float:
+        """W untimed calls, then exactly `steps` calls between two events on
+        the launching stream, barrier + synchronize on both sides; seconds,
+        the max over ranks."""
+        for i in range(warmup):
+            call(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        self.barrier()
+        e0.record(self.stream)
+        for i in range(steps):
+            call(i)
+        e1.record(self.stream)
+        self.barrier()
+        return self.max_over_ranks(e0.elapsed_time(e1) / 1e3)
 
-    # ---- spread of single calls: each call between its own pair of events
-    # (so neighbouring calls do not overlap it), after the timed region ----
-    n_each = max(1, min(args.steps, 2000))
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_each + 1)]
-    barrier()
-    ev[0].record(stream)
-    for i in range(n_each):
-        call(i)
-        ev[i + 1].record(stream)
-    barrier()
-    each_us = sorted(ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(n_each))
-    pct = lambda f: round(each_us[min(n_each - 1, int(f * n_each))], 3)
-    per_call = {"p10": pct(0.10), "p50": pct(0.50), "p90": pct(0.90), "n": n_each, "unit": "us",
-                "how": "each call between its own events, back to back; the headline value is the mean "
-                       "over the timed region"}
+    def per_call(self, call, n) -> dict:
+        """Spread of single calls: each call between its own pair of events,
+        back to back (the events keep neighbouring calls from overlapping it)."""
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+        self.barrier()
+        ev[0].record(self.stream)
+        for i in range(n):
+            call(i)
+            ev[i + 1].record(self.stream)
+        self.barrier()
+        each = sorted(ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(n))
+        pct = lambda f: round(each[min(n - 1, int(f * n))], 3)  # noqa: E731
+        return {"p10": pct(0.10), "p50": pct(0.50), "p90": pct(0.90), "n": n, "unit": "us",
+                "how": "each call between its own events, back to back"}
 
-    # ---- end to end through the C ABI: every step copies its inputs from
-    # pinned host memory (query, block table, lengths; the KV cache lives on
-    # the device) and reads its result back (output and LSE).  As in a
-    # serving loop the copies run on their own streams and overlap the
-    # previous and next steps' kernels: inputs and outputs are double
-    # buffered, and events order each buffer's copy-in, decode and copy-out.
-    hq = (hqv if args.varlen else inp.q).pin_memory()
+
+class Case:
+    """One workload resident on the device, ready to be called."""
+
+    def __init__(self, r: Runner, w, num_splits=None, append=False, varlen=False):
+        from decode_attention_packed_b200 import mxa
+        self.mxa, self.r, self.w = mxa, r, w
+        self.append, self.varlen = append, varlen
+        inp = self.inp = shard_inputs(w, r.rank)
+        dev = r.dev
+        self.q = inp.q.to(dev)
+        self.bt = None if inp.block_table is None else inp.block_table.to(dev)
+        self.sl = inp.cache_seqlens.to(dev)
+        self.pools = [(inp.k_cache.to(dev), inp.v_cache.to(dev))]
+        for _ in range(N_POOLS - 1):
+            self.pools.append((self.pools[0][0].clone(), self.pools[0][1].clone()))
+        self.splits = w.num_splits if num_splits is None else num_splits
+        self.prep = mxa.prepare(self.q, self.pools[0][0], self.bt, max_seqlen_k=inp.max_seqlen_k,
+                                num_splits=self.splits)
+        self.cu = self.hcu = self.hqv = None
+        if varlen:  # the plan above is for q_len queries per row, which bounds every row's count
+            q_lens = np.random.default_rng(w.seed + 77).integers(1, w.q_len + 1, size=w.B)
+            self.hqv, hcu = make_varlen_queries(q_lens, w.Hq, w.D, w.dtype, w.seed + 78)
+            self.q, self.cu = self.hqv.to(dev), hcu.to(dev)
+            self.hcu = hcu.pin_memory()
+        self.out = torch.empty_like(self.q)
+        self.lse = (torch.empty((w.Hq, self.q.shape[0]), dtype=torch.float32, device=dev) if varlen
+                    else torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=dev))
+        self.nbytes = algorithmic_bytes(inp)
+        if append:
+            # the rows' last q_len keys arrive as this step's new tokens: the
+            # call writes them (the same values each step) and attends to all
+            # keys; the new tokens are read and written once more
+            self.nbytes["total"] += 2 * 2 * w.B * w.q_len * w.Hkv * w.D * inp.q.element_size()
+            self.sl_run = (self.sl - w.q_len).clamp(min=0)
+            self.k_new = torch.randn((w.B, w.q_len, w.Hkv, w.D), device=dev).to(self.q.dtype)
+            self.v_new = torch.randn_like(self.k_new)
+        else:
+            self.sl_run = self.sl
+
+    def run(self, i, q, cu, bt, sl, out, lse):
+        mxa, w, prep = self.mxa, self.w, self.prep
+        k, v = self.pools[i % N_POOLS]
+        if self.append:
+            mxa.mxa_decode_fwd_append(q, k, v, self.k_new, self.v_new, bt, sl, prep.params, w.scale, w.causal,
+                                      prep.plan, prep.workspace, out, lse, self.r.stream)
+        elif self.varlen:
+            mxa.mxa_decode_fwd_varlen(q, cu, k, v, bt, sl, prep.params, w.scale, w.causal, prep.plan,
+                                      prep.workspace, out, lse, self.r.stream)
+        else:
+            mxa.mxa_decode_fwd_with_plan(q, k, v, bt, sl, prep.params, w.scale, w.causal, prep.plan,
+                                         prep.workspace, out, lse, self.r.stream)
+
+    def call(self, i):
+        self.run(i, self.q, self.cu, self.bt, self.sl_run, self.out, self.lse)
+
+    def check_clean(self):
+        assert self.mxa.mxa_device_error(True) == self.mxa.MXA_OK, "device-side failure recorded during the bench"
+
+    def roofline(self, per_call_s, peak, peak_kind):
+        achieved = self.nbytes["total"] / per_call_s / 1e9
+        key = (kernel_source_hash(), self.w.name)
+        plain = not (self.append or self.varlen) and self.splits == self.w.num_splits
+        return {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "traffic": MEASURED_TRAFFIC.get(key) if plain else None,
+                "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                else "fallback 6.65 TB/s",
+                "kernel": "mxa_split_kernel (one launch per call; split units merged inside)"}
+
+    def release(self):
+        self.pools = self.q = self.out = self.lse = None
+
+
+def measure(r: Runner, case: Case, args, peak, peak_kind, n_each):
+    """Timed region, spread of single calls and roofline of one workload."""
+    dev_s = r.timed(case.call, args.warmup, args.steps)
+    case.check_clean()
+    per_call_s = dev_s / args.steps
+    kv_gbs = case.nbytes["kv"] / per_call_s / 1e9
+    res = {
+        "us_per_call": round(per_call_s * 1e6, 3),
+        "kv_gbs": round(kv_gbs * r.world, 2),
+        "kv_frac_of_hbm_peak": round(kv_gbs / peak, 4),
+        "kv_bytes_per_call": case.nbytes["kv"],
+        "roofline": case.roofline(per_call_s, peak, peak_kind),
+        "plan": case.prep.plan.as_dict(),
+        "steps": args.steps, "warmup": args.warmup,
+    }
+    # a longer back-to-back run of the same calls, for context
+    n_long = max(args.steps, 2000)
+    long_s = r.timed(case.call, args.warmup, n_long)
+    res["sustained"] = {"us_per_call": round(long_s / n_long * 1e6, 3), "calls": n_long,
+                        "kv_frac_of_hbm_peak": round(case.nbytes["kv"] / (long_s / n_long) / 1e9 / peak, 4)}
+    res["per_call_us"] = r.per_call(case.call, n_each)
+    case.check_clean()
+    return res, dev_s
+
+
+def split_sweep(r: Runner, case: Case, args, peak, n_calls):
+    """µs per call over num_splits (uniform schedule) next to the automatic plan."""
+    mxa = case.mxa
+    rows = []
+    auto = case.prep
+    for s in (0,) + SPLIT_SWEEP:
+        case.prep = mxa.prepare(case.q, case.pools[0][0], case.bt, max_seqlen_k=case.inp.max_seqlen_k,
+                                num_splits=s)
+        t = r.timed(case.call, args.warmup, n_calls) / n_calls
+        case.check_clean()
+        rows.append({"num_splits": s if s else "auto", "schedule": "uniform" if s else "balanced",
+                     "grid": case.prep.plan.grid, "us_per_call": round(t * 1e6, 3),
+                     "kv_frac_of_hbm_peak": round(case.nbytes["kv"] / t / 1e9 / peak, 4)})
+    case.prep = auto
+    return {"calls_per_entry": n_calls, "rows": rows}
+
+
+def e2e(r: Runner, case: Case, args):
+    """End to end through the C ABI: every step copies its inputs from pinned
+    host memory (query, block table, lengths; the KV cache lives on the
+    device) and reads its result back (output and LSE).  As in a serving
+    loop the copies run on their own streams and overlap the previous and
+    next steps' kernels: inputs and outputs are double buffered, and events
+    order each buffer's copy-in, decode and copy-out."""
+    w, inp, dev, stream = case.w, case.inp, r.dev, r.stream
+    hq = (case.hqv if case.varlen else inp.q).pin_memory()
     hbt = None if inp.block_table is None else inp.block_table.pin_memory()
-    hsl = ((inp.cache_seqlens - w.q_len).clamp(min=0) if args.append else inp.cache_seqlens).pin_memory()
+    hsl = ((inp.cache_seqlens - w.q_len).clamp(min=0) if case.append else inp.cache_seqlens).pin_memory()
+    hcu = case.hcu
     h2d = (hq.numel() * hq.element_size() + hsl.numel() * 4 + (0 if hbt is None else hbt.numel() * 4)
            + (0 if hcu is None else hcu.numel() * 4))
-    d2h = out.numel() * out.element_size() + lse.numel() * 4
-    e2e_steps = max(1, min(args.steps, 2000))
+    d2h = case.out.numel() * case.out.element_size() + case.lse.numel() * 4
+    steps = args.steps
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     slots = []
     for _ in range(2):
         slots.append(dict(
-            q=torch.empty_like(q), sl=torch.empty_like(sl), bt=None if bt is None else torch.empty_like(bt),
-            cu=None if cu is None else torch.empty_like(cu),
-            out=torch.empty_like(out), lse=torch.empty_like(lse),
-            hout=torch.empty(out.shape, dtype=out.dtype, pin_memory=True),
-            hlse=torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True),
+            q=torch.empty_like(case.q), sl=torch.empty_like(case.sl),
+            bt=None if case.bt is None else torch.empty_like(case.bt),
+            cu=None if case.cu is None else torch.empty_like(case.cu),
+            out=torch.empty_like(case.out), lse=torch.empty_like(case.lse),
+            hout=torch.empty(case.out.shape, dtype=case.out.dtype, pin_memory=True),
+            hlse=torch.empty(case.lse.shape, dtype=case.lse.dtype, pin_memory=True),
             copied=torch.cuda.Event(), decoded=torch.cuda.Event(), read=torch.cuda.Event()))
     for sd in slots:  # every buffer starts out free
         sd["decoded"].record(stream)
         sd["read"].record(s_out)
 
-    def e2e_step(i):
+    def step(i):
         sd = slots[i % 2]
         with torch.cuda.stream(s_in):
             s_in.wait_event(sd["decoded"])  # the decode two steps back is done with these inputs
@@ -393,7 +482,7 @@ def main():
             sd["copied"].record(s_in)
         stream.wait_event(sd["copied"])
         stream.wait_event(sd["read"])  # the read-back two steps back is done with these outputs
-        run(i, sd["q"], sd["cu"], sd["bt"], sd["sl"], sd["out"], sd["lse"])
+        case.run(i, sd["q"], sd["cu"], sd["bt"], sd["sl"], sd["out"], sd["lse"])
         sd["decoded"].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(sd["decoded"])
@@ -401,21 +490,58 @@ def main():
             sd["hlse"].copy_(sd["lse"], non_blocking=True)
             sd["read"].record(s_out)
 
-    for i in range(min(args.warmup, 50)):
-        e2e_step(i)
-    barrier()
-    torch.cuda.synchronize(dev)
+    for i in range(args.warmup):
+        step(i)
+    r.barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(s_in)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    s_out.wait_event(slots[(e2e_steps - 1) % 2]["read"])
+    for i in range(steps):
+        step(i)
+    s_out.wait_event(slots[(steps - 1) % 2]["read"])
     f1.record(s_out)
-    barrier()
-    torch.cuda.synchronize(dev)
-    e2e_s = max_over_ranks(f0.elapsed_time(f1) / 1e3)
-    for sd in slots:  # the last step's result arrived intact
+    r.barrier()
+    e2e_s = r.max_over_ranks(f0.elapsed_time(f1) / 1e3)
+    for sd in slots:  # the last results arrived intact
         assert torch.equal(sd["hout"], sd["out"].cpu())
+    case.check_clean()
+    return {"value": round(case.nbytes["kv"] * r.world / (e2e_s / steps) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "us_per_step": round(e2e_s / steps * 1e6, 3),
+            "copies": "pinned host buffers on their own streams, double buffered, overlapping the "
+                      "neighbouring steps' kernels"}
+
+
+def main(argv=None):
+    args = parse(argv)
+    world, rank, local = setup_dist(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    r = Runner(world, rank, local)
+    peak, peak_kind = measured_peak()
+    n_each = max(200, min(2000, args.steps))
+    clocks = ClockSampler(local, enabled=not args.no_clocks)
+
+    # ---- the other gated workloads, each in its own timed region ----
+    suite = {}
+    cases = []
+    if args.suite:
+        for name in SUITE:
+            case = Case(r, workload(name))
+            res, _ = measure(r, case, args, peak, peak_kind, n_each)
+            if name == "long_context_split_kv":
+                res["split_sweep"] = split_sweep(r, case, args, peak, n_calls=max(args.steps, 500))
+            res["config"] = workload_config(case.w, case.nbytes, world)
+            suite[name] = res
+            cases.append(case)
+
+    # ---- the headline workload: W warm-up calls, then exactly K timed calls ----
+    w = workload(args.workload)
+    head = Case(r, w, num_splits=args.num_splits, append=args.append, varlen=args.varlen)
+    res, dev_s = measure(r, head, args, peak, peak_kind, n_each)
+    e2e_res = e2e(r, head, args)
+    clk = clocks.stop()
 
     if rank != 0:
         if world > 1:
@@ -423,10 +549,12 @@ def main():
             dist.destroy_process_group()
         return
 
-    peak, peak_kind = measured_peak()
+    if world == 1:  # the oracle on the host cores, after all GPU timing
+        res["cpu_baseline"] = cpu_baseline(head.inp, budget_s=10.0)
+        for case in cases:
+            suite[case.w.name]["cpu_baseline"] = cpu_baseline(case.inp, budget_s=4.0)
     per_call_s = dev_s / args.steps
-    kv_gbs = nbytes["kv"] / per_call_s / 1e9
-    achieved = nbytes["total"] / per_call_s / 1e9
+    kv_gbs = head.nbytes["kv"] / per_call_s / 1e9
     line = {
         "metric": METRIC,
         "value": round(kv_gbs * world, 2),
@@ -434,35 +562,33 @@ def main():
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(dev_s / args.steps * 1e3, 5),
-        "us_per_call": round(per_call_s * 1e6, 3),
-        "per_call_us": per_call,
-        "kv_frac_of_hbm_peak": round(kv_gbs / peak, 4),
+        "ms_per_step": round(per_call_s * 1e3, 5),
+        "us_per_call": res["us_per_call"],
+        "per_call_us": res["per_call_us"],
+        "sustained": res["sustained"],
+        "kv_frac_of_hbm_peak": res["kv_frac_of_hbm_peak"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic",
-        "config": dict(workload_config(w, nbytes, world), append=bool(args.append),
+        "config": dict(workload_config(w, head.nbytes, world), append=bool(args.append),
                        **({"varlen": {"q_lens": "U{1..%d} per row, seeded" % w.q_len,
-                                      "total_q": int(q.shape[0])}} if args.varlen else {})),
-        "plan": prep.plan.as_dict(),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4),
-                     "traffic": MEASURED_TRAFFIC.get(kernel_source_hash())
-                     if w.name == DEFAULT_WORKLOAD and not (args.append or args.varlen) else None,
-                     "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                     else "fallback 6.65 TB/s",
-                     "kernel": "mxa_split_kernel (one launch per call; split units merged inside)"},
-        "e2e": {"value": round(nbytes["kv"] * world / (e2e_s / e2e_steps) / 1e9, 2), "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "copies": "pinned host buffers on their own streams, double buffered, overlapping the "
-                          "neighbouring steps' kernels"},
-        "gpu_launches": args.steps * launches_per_call,
+                                      "total_q": int(head.q.shape[0])}} if args.varlen else {})),
+        "plan": res["plan"],
+        "roofline": res["roofline"],
+        "e2e": e2e_res,
+        "gpu_launches": args.steps,
         "clocks": clk,
     }
-    if world == 1:
-        line["cpu_baseline"] = cpu_baseline(inp)
+    if "cpu_baseline" in res:
+        line["cpu_baseline"] = res["cpu_baseline"]
+    if suite:
+        line["workloads"] = suite
+        fracs = {name: v["kv_frac_of_hbm_peak"] for name, v in suite.items()}
+        fracs[w.name] = res["kv_frac_of_hbm_peak"]
+        line["gate"] = {"kv_frac_of_hbm_peak": fracs, "target": 0.70,
+                        "all_met": all(f >= 0.70 for f in fracs.values())}
     print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -113,6 +113,7 @@ mxa_status_t prepare_decode(const void *q, const void *k_cache, const void *v_ca
   L.k_new = L.v_new = nullptr;
   L.cu_q = nullptr;
   L.total_q = 0;
+  L.out_f32 = 0;
   return MXA_OK;
 }
 
@@ -255,6 +256,29 @@ mxa_status_t mxa_decode_fwd_with_plan(const void *q, const void *k_cache, const 
   return launch_decode(L, static_cast<cudaStream_t>(stream));
 }
 
+mxa_status_t mxa_decode_fwd_f32out(const void *q, const void *k_cache, const void *v_cache,
+                                   const int32_t *block_table, const int32_t *cache_seqlens,
+                                   const mxa_decode_params_t *p, float scale, int causal, const mxa_plan_t *plan,
+                                   void *workspace, size_t workspace_bytes, float *out, float *lse,
+                                   void *stream) {
+  DecodeLaunch L;
+  mxa_status_t st = prepare_decode(q, k_cache, v_cache, block_table, cache_seqlens, p, scale, causal, plan,
+                                   workspace, workspace_bytes, out, lse, &L);
+  if (st != MXA_OK || p->B == 0) return st;
+  L.out_f32 = 1;
+  return launch_decode(L, static_cast<cudaStream_t>(stream));
+}
+
+size_t mxa_decode_workspace_size(const mxa_decode_params_t *p, int num_splits) {
+  if (num_splits < 0) return SIZE_MAX;
+  mxa_plan_t plan;
+  // a uniform plan does not depend on the device; the automatic one is sized
+  // for the current device's SMs
+  const int sm_count = num_splits > 0 ? 1 : 0;
+  if (mxa_plan(p, num_splits, sm_count, &plan) != MXA_OK) return SIZE_MAX;
+  return plan.workspace_bytes;
+}
+
 mxa_status_t mxa_decode_fwd_append(const void *q, void *k_cache, void *v_cache, const void *k_new,
                                    const void *v_new, const int32_t *block_table, const int32_t *cache_seqlens,
                                    const mxa_decode_params_t *p, float scale, int causal, const mxa_plan_t *plan,
@@ -324,8 +348,8 @@ mxa_status_t mxa_device_error(int reset) {
   int flags = 0;
   mxa_status_t st = read_device_error(reset, &flags);
   if (st != MXA_OK) return st;
-  if (flags & ~kErrBadPage) return MXA_ERR_TIMEOUT;
-  return flags ? MXA_ERR_INVALID_ARG : MXA_OK;  // an appended token's page id was outside the pool
+  if (flags & ~kErrInputMask) return MXA_ERR_TIMEOUT;
+  return flags ? MXA_ERR_INVALID_ARG : MXA_OK;  // inputs outside the contract, confined and clamped
 }
 
 }  // extern "C"

@@ -19,12 +19,18 @@ constexpr int kMaxBalancedRows = 12288;                 // balanced schedule sca
 constexpr int kMaxUnitCost = 64;
 
 // Device-side failure record (bit flags), read back by mxa_device_error():
-// bounded waits that ran out, a misaligned shared-memory base, and
-// block-table entries outside the pool (read as zeros; appended tokens there
-// not written).
+// bounded waits that ran out and a misaligned shared-memory base (reported
+// as a timeout), and inputs that break the call's contract, which the kernel
+// confines to the buffers and reports as an invalid argument: block-table
+// entries outside the pool (read as zeros; appended tokens there not
+// written), lengths outside [0, max_seqlen_k] (clamped into that range), and
+// query offsets that do not run from 0 up to total_q by steps of at most
+// q_len (clamped likewise).
 enum : int {
-  kErrWaitFull = 1, kErrWaitEmpty = 2, kErrWaitQ = 4, kErrAlign = 8, kErrDrain = 16, kErrBadPage = 32
+  kErrWaitFull = 1, kErrWaitEmpty = 2, kErrWaitQ = 4, kErrAlign = 8, kErrDrain = 16, kErrBadPage = 32,
+  kErrBadLen = 64, kErrBadOffsets = 128
 };
+constexpr int kErrInputMask = kErrBadPage | kErrBadLen | kErrBadOffsets;
 
 // Fixed cost of a unit in the balanced schedule, in KV blocks: the work a
 // unit needs besides streaming its keys (the cross-warp merge, the output

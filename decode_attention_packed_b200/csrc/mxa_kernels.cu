@@ -44,8 +44,10 @@ __device__ int g_mxa_err = 0;
 
 constexpr float kLn2 = 0.6931471805599453f;
 
-__device__ __forceinline__ int clamp_len(int L, int max_len) {
-  return L < 0 ? 0 : (L > max_len ? max_len : L);
+// A row's key count clamped into [0, max_len]; L is taken in 64 bits so that
+// a length plus the appended tokens cannot overflow.
+__device__ __forceinline__ int clamp_len(long long L, int max_len) {
+  return L < 0 ? 0 : (L > max_len ? max_len : (int)L);
 }
 
 __device__ __forceinline__ uint32_t bar_addr(const uint8_t *smem, int D, int i) {
@@ -77,7 +79,7 @@ struct Cursor {
   long long x, end;
   long long per_cta;  // positions per CTA range (balanced schedule)
   int L, nb;          // length and blocks of row b
-  int L_next;         // prefetched length of row b + 1
+  long long L_next;   // prefetched length of row b + 1 (with the appended tokens; not clamped yet)
   int rtb;            // row tiles of row b: its units are hr < Hkv * rtb
   int q0, qn;         // row b's queries: first packed token, count
   int q0_next, qn_next;  // prefetched queries of row b + 1 (per-row queries only)
@@ -129,7 +131,7 @@ __device__ __forceinline__ void cursor_enter_row(Cursor &c, const DecodeArgs &a,
     c.q0 = c.b * a.q_len;
     c.qn = a.q_len;
   }
-  c.L_next = c.b + 1 < a.B ? a.seqlens[c.b + 1] + a.len_add : 0;  // consumed a segment later
+  c.L_next = c.b + 1 < a.B ? (long long)a.seqlens[c.b + 1] + a.len_add : 0;  // consumed a segment later
 }
 
 // The segment at the cursor (a contiguous block range of one unit); the
@@ -171,7 +173,7 @@ __device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
         cursor_enter_row<D, kVarlen>(c, a, clamp_len(c.L_next, a.max_seqlen_k));
         while (c.nb == 0 && c.b + 1 < a.B) {  // rows without keys (or queries) hold no units
           ++c.b;
-          cursor_enter_row<D, kVarlen>(c, a, clamp_len(a.seqlens[c.b] + a.len_add, a.max_seqlen_k));
+          cursor_enter_row<D, kVarlen>(c, a, clamp_len((long long)a.seqlens[c.b] + a.len_add, a.max_seqlen_k));
         }
       } else {
         c.end = c.x;
@@ -211,7 +213,7 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
     c.b = u / HR;
     c.hr = u % HR;
     row_queries<kVarlen>(a, c.b, c.q0, c.qn);
-    c.L = clamp_len(a.seqlens[c.b] + a.len_add, a.max_seqlen_k);
+    c.L = clamp_len((long long)a.seqlens[c.b] + a.len_add, a.max_seqlen_k);
     c.nb = (c.L + T - 1) / T;
     if (kVarlen && c.hr % a.RT >= row_tiles(a, c.qn)) c.nb = 0;  // a tile past the row's queries
     const int beg = si * a.chunk_blocks, end = min(beg + a.chunk_blocks, c.nb);
@@ -227,7 +229,7 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
   const int lo = min(lane * chunk, a.B), hi = min(lo + chunk, a.B);
   int sum = 0;
   for (int i = lo; i < hi; ++i) {
-    const int L = clamp_len(a.seqlens[i] + a.len_add, a.max_seqlen_k);
+    const int L = clamp_len((long long)a.seqlens[i] + a.len_add, a.max_seqlen_k);
     lens[i] = L;
     const int nb = (L + T - 1) / T;
     int w = nb > 0 ? nb + V : 0;  // positions of one unit of row i
@@ -496,7 +498,7 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
         // Tokens this call appends that fall in this block go into the cache
         // first (this unit's KV head), and are fenced against the loads below.
         if constexpr (kAppend) {
-          const int n0 = new0 < 0 ? 0 : new0, n1 = min(new0 + a.len_add, seg.L);
+          const int n0 = new0 < 0 ? 0 : new0, n1 = (int)min((long long)new0 + a.len_add, (long long)seg.L);
           const int p0 = max(n0, tok0), p1 = min(n1, tok0 + T);
           if (p1 > p0) {
             write_new_tokens(seg, win, new0, p0, p1);
@@ -848,6 +850,19 @@ __device__ void math_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lan
 // Epilogue warp
 // ---------------------------------------------------------------------------
 
+// D / 32 consecutive float32 values of packed row `rr` into the rows at
+// shared address `stage` (row pitch D * 4 bytes): partial results, and the
+// output when it is float32.
+template <int D>
+__device__ __forceinline__ void stage_f32_vec(uint8_t *smem, uint32_t stage, int rr, int col, const float *v) {
+  float *dst = reinterpret_cast<float *>(smem + (stage - smem_addr(smem))) + rr * D + col;
+  if constexpr (D / 32 == 4) {
+    *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+  } else {
+    *reinterpret_cast<float2 *>(dst) = make_float2(v[0], v[1]);
+  }
+}
+
 // D / 32 consecutive values of packed row `rr`, rounded to the output type,
 // into the staging rows at shared address `stage` (row pitch D * 2 bytes).
 // A plain store, so the compiler may overlap it with the loads of other rows.
@@ -868,12 +883,13 @@ __device__ __forceinline__ void stage_out_vec(uint8_t *smem, uint32_t stage, int
 template <int D>
 __device__ __forceinline__ void store_out_rows(const DecodeArgs &a, int q0, int h, int rt, int rows,
                                                uint32_t stage) {
+  const int es = a.out_f32 ? 4 : 2;  // bytes per output element
   int r = 0;
   while (r < rows) {
     const int m = rt * kRowsPerTile + r, t = m / a.G, g = m % a.G;
     const int r_end = min(rows, (t + 1) * a.G - rt * kRowsPerTile);
-    uint16_t *dst = reinterpret_cast<uint16_t *>(a.out) + ((size_t)(q0 + t) * a.Hq + (size_t)h * a.G + g) * D;
-    bulk_store(dst, stage + (uint32_t)(r * D * 2), (uint32_t)((r_end - r) * D * 2));
+    uint8_t *dst = reinterpret_cast<uint8_t *>(a.out) + ((size_t)(q0 + t) * a.Hq + (size_t)h * a.G + g) * D * es;
+    bulk_store(dst, stage + (uint32_t)(r * D * es), (uint32_t)((r_end - r) * D * es));
     r = r_end;
   }
 }
@@ -888,11 +904,12 @@ __device__ void write_empty_unit(const DecodeArgs &a, int unit, int lane) {
   else row_queries<false>(a, b, q0, qn);
   if (rt >= row_tiles(a, qn)) return;  // the same for every lane
   const int rows = tile_rows(a, qn, rt);
-  uint16_t *out = reinterpret_cast<uint16_t *>(a.out);
   for (int i = lane; i < rows * D; i += 32) {
     const int rr = i / D, d = i % D;
     const int m = rt * kRowsPerTile + rr, t = m / a.G, g = m % a.G;
-    out[((size_t)(q0 + t) * a.Hq + (size_t)h * a.G + g) * D + d] = 0;  // +0 in fp16 and bf16
+    const size_t e = ((size_t)(q0 + t) * a.Hq + (size_t)h * a.G + g) * D + d;
+    if (a.out_f32) reinterpret_cast<float *>(a.out)[e] = 0.f;
+    else reinterpret_cast<uint16_t *>(a.out)[e] = 0;  // +0 in fp16 and bf16
   }
   if (a.lse != nullptr) {
     for (int rr = lane; rr < rows; rr += 32) {
@@ -901,6 +918,23 @@ __device__ void write_empty_unit(const DecodeArgs &a, int unit, int lane) {
     }
   }
   __syncwarp();
+}
+
+// Check the inputs of batch row b against the call's contract and record a
+// breach: a length outside [0, max_seqlen_k] (the kernels clamp it into that
+// range), and with per-row queries offsets that do not rise from 0 to
+// total_q by steps of at most q_len (clamped likewise).  Every access stays
+// inside the buffers either way; the record tells the caller that the
+// result answers clamped inputs, not the ones passed.
+__device__ __forceinline__ void check_row_inputs(const DecodeArgs &a, int b) {
+  int bad = 0;
+  const int L = a.seqlens[b];
+  if (L < 0 || L > a.max_seqlen_k) bad |= kErrBadLen;
+  if (a.cu_q != nullptr) {
+    const int s = a.cu_q[b], e = a.cu_q[b + 1];
+    if (e < s || (long long)e - s > a.q_len || (b == 0 && s != 0) || (b == a.B - 1 && e != a.total_q)) bad |= kErrBadOffsets;
+  }
+  if (bad) atomicOr(&g_mxa_err, bad);
 }
 
 // Room for partial rows in a landing zone that is a whole ring stage; its
@@ -1057,7 +1091,10 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
   __syncwarp();  // every lane is done with the landing zone, which may be the staging buffer
 #pragma unroll
   for (int rr = 0; rr < NR; ++rr)
-    if (rr < rows) stage_out_vec<D, kBf16>(smem, ostage, rr, col, acc[rr]);
+    if (rr < rows) {
+      if (a.out_f32) stage_f32_vec<D>(smem, ostage, rr, col, acc[rr]);
+      else stage_out_vec<D, kBf16>(smem, ostage, rr, col, acc[rr]);
+    }
   fence_proxy_async_smem();  // staged rows are read by the bulk stores
   __syncwarp();
   if (lane == 0) {
@@ -1098,13 +1135,17 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
   grid_dependency_wait();
 
   // Units of rows with L_b = 0 hold no KV block; one CTA per unit writes
-  // their empty result.
+  // their empty result.  The CTA of a row's first unit also checks the
+  // row's inputs against the call's contract.
   if (a.schedule == MXA_SCHED_BALANCED) {
-    for (int u = blockIdx.x; u < a.units; u += gridDim.x)
-      if (clamp_len(a.seqlens[u / HR] + a.len_add, a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, lane);
+    for (int u = blockIdx.x; u < a.units; u += gridDim.x) {
+      if (u % HR == 0 && lane == 0) check_row_inputs(a, u / HR);
+      if (clamp_len((long long)a.seqlens[u / HR] + a.len_add, a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, lane);
+    }
   } else if (blockIdx.x % a.splits == 0) {
     const int u = blockIdx.x / a.splits;
-    if (clamp_len(a.seqlens[u / HR] + a.len_add, a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, lane);
+    if (u % HR == 0 && lane == 0) check_row_inputs(a, u / HR);
+    if (clamp_len((long long)a.seqlens[u / HR] + a.len_add, a.max_seqlen_k) == 0) write_empty_unit<D>(a, u, lane);
   }
 
   // Tag the arrival counters of this CTA's split units with this launch's
@@ -1238,19 +1279,13 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
       merge_now = all_here && sg.n_pieces <= min(lse_slots, (int)(land_rows / pbytes));
       __syncwarp();  // every lane has read the stage before it may become the landing zone
       dst_rows = merge_now ? land + (uint32_t)own * pbytes : ostage;
+      // 16-bit output rows, or float32 rows (a partial result, or a float32 output)
+      const bool rows16 = sg.kind == 0 && !a.out_f32;
 #pragma unroll
       for (int rr = 0; rr < NR; ++rr) {
         if (rr < rows) {
-          if (sg.kind == 0) {
-            stage_out_vec<D, kBf16>(smem, ostage, rr, col, acc[rr]);
-          } else {  // fp32 partial rows, pitch D * 4 bytes
-            float *dst = reinterpret_cast<float *>(smem + (dst_rows - smem_addr(smem))) + rr * D + col;
-            if constexpr (VEC == 4) {
-              *reinterpret_cast<float4 *>(dst) = make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
-            } else {
-              *reinterpret_cast<float2 *>(dst) = make_float2(acc[rr][0], acc[rr][1]);
-            }
-          }
+          if (rows16) stage_out_vec<D, kBf16>(smem, ostage, rr, col, acc[rr]);
+          else stage_f32_vec<D>(smem, dst_rows, rr, col, acc[rr]);
         }
       }
     };
@@ -1555,6 +1590,7 @@ mxa_status_t launch_typed(const DecodeLaunch &L, cudaStream_t stream) {
   a.k_cache_w = static_cast<uint16_t *>(const_cast<void *>(L.k_cache));
   a.v_cache_w = static_cast<uint16_t *>(const_cast<void *>(L.v_cache));
   a.epoch = next_epoch();
+  a.out_f32 = L.out_f32;
   if (plan.workspace_bytes > 0) {
     uint8_t *ws = static_cast<uint8_t *>(L.workspace);
     a.counters = reinterpret_cast<unsigned long long *>(ws);

@@ -48,6 +48,7 @@ struct DecodeArgs {
   uint16_t *k_cache_w;         // the caches, written at the appended positions
   uint16_t *v_cache_w;
   unsigned int epoch;          // tags this launch's arrival counts
+  int out_f32;                 // 1: out holds float32 (the value before its one rounding)
 };
 
 // Everything launch_decode needs; pointers are device pointers.
@@ -65,6 +66,7 @@ struct DecodeLaunch {
   const void *k_new, *v_new;  // [B, q_len, Hkv, D] when len_add > 0
   const int32_t *cu_q;        // varlen: [B + 1] query offsets (null: q_len queries per row)
   int total_q;                // varlen: packed query tokens
+  int out_f32;                // out is float32 instead of the input type
 };
 
 // Launch the split kernel (split units are merged inside it).

@@ -30,7 +30,10 @@ MXA_SCHED_UNIFORM, MXA_SCHED_BALANCED = 0, 1
 EXPORTED = ("mxa_status_string", "mxa_should_pack_gqa", "mxa_num_splits_heuristic", "mxa_plan",
             "mxa_plan_balanced",
             "mxa_decode_fwd", "mxa_decode_fwd_with_plan", "mxa_combine", "mxa_device_error",
-            "mxa_decode_fwd_noalloc", "mxa_decode_fwd_append", "mxa_decode_fwd_varlen")
+            "mxa_decode_fwd_noalloc", "mxa_decode_fwd_append", "mxa_decode_fwd_varlen",
+            "mxa_decode_fwd_f32out", "mxa_decode_workspace_size")
+
+SIZE_MAX = ctypes.c_size_t(-1).value
 
 
 class mxa_decode_params_t(ctypes.Structure):
@@ -70,6 +73,10 @@ _lib.mxa_decode_fwd_with_plan.argtypes = [_P, _P, _P, _P, _P, ctypes.POINTER(mxa
                                           ctypes.c_float, _I, ctypes.POINTER(mxa_plan_t), _P,
                                           ctypes.c_size_t, _P, _P, _P]
 _lib.mxa_decode_fwd_with_plan.restype = _I
+_lib.mxa_decode_fwd_f32out.argtypes = _lib.mxa_decode_fwd_with_plan.argtypes
+_lib.mxa_decode_fwd_f32out.restype = _I
+_lib.mxa_decode_workspace_size.argtypes = [ctypes.POINTER(mxa_decode_params_t), _I]
+_lib.mxa_decode_workspace_size.restype = ctypes.c_size_t
 _lib.mxa_decode_fwd_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(mxa_decode_params_t),
                                        ctypes.c_float, _I, ctypes.POINTER(mxa_plan_t), _P, ctypes.c_size_t,
                                        _P, _P, _P]
@@ -156,6 +163,25 @@ def mxa_decode_fwd_with_plan(q, k_cache, v_cache, block_table, cache_seqlens, pa
                                          int(causal), ctypes.byref(plan), _ptr(workspace), ws_bytes,
                                          _ptr(out), _ptr(lse), _stream(stream)),
            "mxa_decode_fwd_with_plan")
+
+
+def mxa_decode_fwd_f32out(q, k_cache, v_cache, block_table, cache_seqlens, params, scale, causal,
+                          plan, workspace, out, lse, stream=None) -> None:
+    """As mxa_decode_fwd_with_plan with a float32 `out`: O before its rounding
+    to the input type."""
+    if out.dtype != torch.float32:
+        raise TypeError("mxa_decode_fwd_f32out writes a float32 out")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.mxa_decode_fwd_f32out(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                      _ptr(cache_seqlens), ctypes.byref(params), float(scale),
+                                      int(causal), ctypes.byref(plan), _ptr(workspace), ws_bytes,
+                                      _ptr(out), _ptr(lse), _stream(stream)),
+           "mxa_decode_fwd_f32out")
+
+
+def mxa_decode_workspace_size(params: mxa_decode_params_t, num_splits: int = 0) -> int:
+    """Workspace bytes of mxa_plan(params, num_splits); SIZE_MAX when refused."""
+    return int(_lib.mxa_decode_workspace_size(ctypes.byref(params), int(num_splits)))
 
 
 def mxa_decode_fwd_append(q, k_cache, v_cache, k_new, v_new, block_table, cache_seqlens, params, scale,
@@ -254,24 +280,32 @@ def prepare(q, k_cache, block_table, *, max_seqlen_k=None, num_splits=0, plan=No
 
 def decode(q, k_cache, v_cache, block_table, cache_seqlens, *, scale=None, causal=False,
            num_splits=0, max_seqlen_k=None, out=None, lse=None, prepared: Optional[Prepared] = None,
-           return_lse=True, stream=None, k_new=None, v_new=None):
+           return_lse=True, stream=None, k_new=None, v_new=None, out_dtype=None):
     """out [B, q_len, Hq, D] (and lse [B, Hq, q_len] fp32) for one decode step.
 
     With k_new / v_new [B, q_len, Hkv, D] the step first writes them into the
     cache at positions cache_seqlens[b] + t and attends to cache_seqlens[b] +
-    q_len keys; max_seqlen_k must then bound those lengths."""
+    q_len keys; max_seqlen_k must then bound those lengths.  out_dtype =
+    torch.float32 returns O before its rounding to q's type
+    (mxa_decode_fwd_f32out)."""
     if scale is None:
         scale = q.shape[-1] ** -0.5
     if prepared is None:
         prepared = prepare(q, k_cache, block_table, max_seqlen_k=max_seqlen_k, num_splits=num_splits)
+    f32 = out_dtype == torch.float32 or (out is not None and out.dtype == torch.float32)
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device) if f32 else torch.empty_like(q)
     if lse is None and return_lse:
         B, q_len, Hq, _ = q.shape
         lse = torch.empty((B, Hq, q_len), dtype=torch.float32, device=q.device)
     if (k_new is None) != (v_new is None):
         raise ValueError("k_new and v_new go together")
-    if k_new is None:
+    if f32:
+        if k_new is not None:
+            raise ValueError("a float32 output is not offered with k_new / v_new")
+        mxa_decode_fwd_f32out(q, k_cache, v_cache, block_table, cache_seqlens, prepared.params, scale, causal,
+                              prepared.plan, prepared.workspace, out, lse, stream)
+    elif k_new is None:
         mxa_decode_fwd_with_plan(q, k_cache, v_cache, block_table, cache_seqlens, prepared.params, scale,
                                  causal, prepared.plan, prepared.workspace, out, lse, stream)
     else:

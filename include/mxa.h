@@ -87,6 +87,9 @@ typedef enum { MXA_SCHED_UNIFORM = 0, MXA_SCHED_BALANCED = 1 } mxa_schedule_t;
  *                and values read as zeros, and mxa_device_error reports
  *                MXA_ERR_INVALID_ARG)
  *   cache_seqlens[B] int32: number of valid keys L_b, 0 <= L_b <= max_seqlen_k
+ *                (a length outside that range is clamped into it, so no access
+ *                leaves the buffers, and mxa_device_error reports
+ *                MXA_ERR_INVALID_ARG)
  *   out          [B, q_len, Hq, D]                 dtype
  *   lse          [B, Hq, q_len]                    float32, natural log
  * Query head h reads KV head h / (Hq / Hkv).
@@ -177,6 +180,19 @@ MXA_API mxa_status_t mxa_plan(const mxa_decode_params_t *params, int num_splits,
 MXA_API mxa_status_t mxa_plan_balanced(const mxa_decode_params_t *params, int grid, int sm_count,
                                        mxa_plan_t *plan);
 
+/* Bytes of device workspace that a run of mxa_plan(params, num_splits, ...)
+ * needs: the first phase of the two-phase call ("SmallQ FlashAttention
+ * (Vector)" README, section aclnn API 调用: ...GetWorkspaceSize, then the
+ * operator with that workspace).  0 means no workspace is needed.
+ *   num_splits > 0 : the UNIFORM plan with that many splits (a pure host
+ *                    computation: the size does not depend on the device);
+ *   num_splits == 0: the automatic plan for the current CUDA device.
+ * Returns SIZE_MAX when mxa_plan would refuse the arguments (a NULL or
+ * inconsistent params, an unsupported shape, num_splits < 0) or, for the
+ * automatic plan, when no CUDA device can be queried.  mxa_plan returns the
+ * same number in plan.workspace_bytes, with the rest of the plan. */
+MXA_API size_t mxa_decode_workspace_size(const mxa_decode_params_t *params, int num_splits);
+
 /* Decode attention, one call: plan (num_splits as in mxa_plan, on the
  * current device) and run.
  *   q, k_cache, v_cache, block_table, cache_seqlens : device, read only
@@ -208,6 +224,24 @@ MXA_API mxa_status_t mxa_decode_fwd_with_plan(const void *q, const void *k_cache
                                       const mxa_plan_t *plan, void *workspace,
                                       size_t workspace_bytes, void *out, float *lse,
                                       void *stream);
+
+/* As mxa_decode_fwd_with_plan, but `out` receives O in float32: the
+ * normalised output before its one rounding to the input type (the
+ * precision policy of the "SmallQ FlashAttention (Vector)" README, section
+ * 精度策略: fp32 dot products and accumulation, and a single rounding of
+ * acc * (1 / rowSum) at the end).  The same kernels and plan run; only the
+ * output rows are stored as float32.  Uses: checking the computation itself
+ * against a reference at a tolerance tighter than a 16-bit output's own
+ * rounding, and callers that merge the result with partial results from
+ * elsewhere (another cache segment, another GPU) through mxa_combine, which
+ * takes exactly this float32 O with its LSE.
+ *   out : device [B, q_len, Hq, D] float32 (written in full)
+ * Other arguments and errors as mxa_decode_fwd_with_plan. */
+MXA_API mxa_status_t mxa_decode_fwd_f32out(const void *q, const void *k_cache, const void *v_cache,
+                                           const int32_t *block_table, const int32_t *cache_seqlens,
+                                           const mxa_decode_params_t *params, float scale, int causal,
+                                           const mxa_plan_t *plan, void *workspace, size_t workspace_bytes,
+                                           float *out, float *lse, void *stream);
 
 /* Append the new tokens' keys and values to the cache, then decode, in one
  * call: the k / v arguments of flash_attn_with_kvcache next to cache_seqlens
@@ -252,10 +286,12 @@ MXA_API mxa_status_t mxa_decode_fwd_append(const void *q, void *k_cache, void *v
  * Row b with q_b = cu[b+1] - cu[b] queries: non-causal, every query sees L_b
  * keys; causal, query t sees the first L_b - q_b + t + 1 (its queries are
  * the row's last q_b cache entries).  A row with q_b = 0 writes nothing.
- * Offsets are read on the device and not checked there against these rules:
- * out-of-range values are clamped into [0, total_q] and a row's count to
- * params->q_len, so that no access leaves the buffers, but the result of
- * such a call is unspecified.  Other arguments and errors as
+ * Offsets are read on the device.  Offsets that break these rules (not
+ * starting at 0, decreasing, ending away from total_q, or a count above
+ * params->q_len) are clamped into [0, total_q] and a row's count to
+ * params->q_len, so that no access leaves the buffers; the result of such a
+ * call is unspecified, and mxa_device_error reports MXA_ERR_INVALID_ARG.
+ * Other arguments and errors as
  * mxa_decode_fwd_with_plan; MXA_ERR_INVALID_ARG for a NULL or misaligned
  * cu_seqlens_q or total_q < 0. */
 MXA_API mxa_status_t mxa_decode_fwd_varlen(const void *q, const int32_t *cu_seqlens_q, int total_q,
@@ -276,7 +312,12 @@ MXA_API mxa_status_t mxa_decode_fwd_varlen(const void *q, const int32_t *cu_seql
  * same kernels, but keeps the split results in one fixed 16 MiB array inside
  * the library.  It calls no allocator at all.
  *  - The array is part of the library's device image: every GPU that loads
- *    the library holds those 16 MiB until the process exits.
+ *    the library's device code holds those 16 MiB until the process exits.
+ *    Under CUDA's lazy module loading (the default since CUDA 12) that image,
+ *    array included, is loaded at the first call on each device that needs
+ *    it, not when the library is opened: a caller that reserves its memory
+ *    up front makes one call first (any shape whose plan splits, e.g. the
+ *    decode it is about to run) and reserves after it.
  *  - A plan that needs more scratch than 16 MiB is refused with
  *    MXA_ERR_WORKSPACE (use mxa_decode_fwd with your own workspace then).
  *  - The first call on each device looks up the array's device address
@@ -310,11 +351,19 @@ MXA_API mxa_status_t mxa_combine(const float *o_part, const float *lse_part, int
 
 /* Synchronise the current device and report whether any kernel of this
  * library recorded a device-side failure since the last reset: MXA_OK;
- * MXA_ERR_TIMEOUT if a bounded wait ran out; else MXA_ERR_INVALID_ARG if a
- * block-table entry that a kernel used lay outside [0, num_pages) (its keys
- * read as zeros; an appended token there was not written); MXA_ERR_CUDA if
- * the device or the synchronisation itself failed.
- * reset != 0 clears the record. */
+ * MXA_ERR_TIMEOUT if a bounded wait ran out; else MXA_ERR_INVALID_ARG if
+ * device-resident inputs broke the call's contract (the kernels confine the
+ * call to its buffers and go on): a block-table entry that a kernel used lay
+ * outside [0, num_pages) (its keys read as zeros; an appended token there
+ * was not written), a cache_seqlens value lay outside [0, max_seqlen_k]
+ * (clamped), or varlen query offsets broke their rules (clamped);
+ * MXA_ERR_CUDA if the device or the synchronisation itself failed.
+ * reset != 0 clears the record.
+ * After MXA_ERR_TIMEOUT a split unit's arrival counter in the workspace (or
+ * in mxa_decode_fwd_noalloc's array) may be left mid-count.  Every launch
+ * normally tags the counters with a fresh epoch, so a direct call recovers
+ * by itself; a captured CUDA graph replays one epoch, so zero the workspace
+ * (or recapture the graph) before replaying it after a timeout. */
 MXA_API mxa_status_t mxa_device_error(int reset);
 
 #ifdef __cplusplus

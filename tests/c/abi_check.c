@@ -15,6 +15,10 @@ int main(void) {
          plan.grid, plan.units, plan.unit_cost, plan.needs_combine, plan.workspace_bytes);
   st = mxa_plan(&p, 4, 148, &plan);
   printf("uniform %d schedule %d grid %d splits %d\n", (int)st, plan.schedule, plan.grid, plan.num_splits);
+  /* the first phase of the two-phase call, from C: the uniform plan's size
+   * (a host computation) and a refusal */
+  printf("wsize %zu %zu %d\n", mxa_decode_workspace_size(&p, 4), plan.workspace_bytes,
+         mxa_decode_workspace_size(&p, -1) == (size_t)-1);
   printf("pack %d %d\n", mxa_should_pack_gqa(0, 1, 4, 64), mxa_should_pack_gqa(0, 128, 1, 64));
   printf("splits %d %d\n", mxa_num_splits_heuristic(16, 148, 296, 128, 128, 0, 1, 8388608.0),
          mxa_num_splits_heuristic(256, 148, 296, 32, 64, 0, 1, 1048576.0));

@@ -59,3 +59,16 @@ def test_cuda_arm_fails_loudly_without_a_gpu():
     r = run_bench("--steps", "1", "--warmup", "1", "--no-clocks", timeout=300)
     assert r.returncode != 0
     assert not [ln for ln in r.stdout.splitlines() if ln.strip().startswith("{")]
+
+
+def test_default_run_is_the_headline_with_the_suite():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    a = bench.parse([])
+    assert a.workload == bench.HEADLINE == "ragged_varlen" and a.suite and a.gpus == 1
+    assert (a.steps, a.warmup) == (20, 5)
+    assert set(bench.SUITE) == {"gqa_decode", "spec_mtp_small_q", "long_context_split_kv"}
+    b = bench.parse(["--workload", "gqa_decode"])
+    assert b.workload == "gqa_decode" and not b.suite
+    assert not bench.parse(["--no-suite"]).suite

@@ -33,6 +33,9 @@ def test_c_caller_gets_the_python_binding_plan(abi_check):
     assert abi_check["plan"] == want
     u = mxa.mxa_plan(p, 4, sm_count=148)
     assert abi_check["uniform"] == f"{mxa.MXA_OK} schedule {u.schedule} grid {u.grid} splits {u.num_splits}"
+    # mxa_decode_workspace_size agrees with the plan mxa_plan returns, and refuses num_splits < 0
+    assert u.workspace_bytes > 0
+    assert abi_check["wsize"] == f"{u.workspace_bytes} {u.workspace_bytes} 1"
 
 
 def test_c_caller_gets_the_rules_and_refusals(abi_check):

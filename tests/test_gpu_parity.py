@@ -335,3 +335,41 @@ def test_a_page_id_outside_the_pool_reads_as_zeros_and_is_reported(bad_page):
                            scale=w.scale, causal=False)
     assert_out_close(out.cpu(), ro, w.dtype)
     assert_lse_close(lse.cpu(), rl)
+
+
+@pytest.mark.parametrize("bad_len", [70, -3, 2**31 - 1, -2**31])
+def test_a_length_outside_the_bound_is_clamped_and_reported(bad_len):
+    # row 1's length lies outside [0, max_seqlen_k = 64]: the call must stay
+    # inside its buffers, attend to the clamped length (64 keys, or none),
+    # leave the other rows alone, and report the breach
+    w = Workload(name="badlen", B=3, q_len=1, Hq=8, Hkv=2, D=128, dtype="bf16", page_size=16, causal=False,
+                 lengths="list:40,70,33", seed=546)
+    inp = make_inputs(w)  # a block table wide enough for 70 keys
+    d = "cuda"
+    sl = inp.cache_seqlens.clone()
+    sl[1] = bad_len
+    pad = 64
+    out_buf = torch.full((3 + 2 * pad, 1, 8, 128), 7.0, dtype=torch.bfloat16, device=d)
+    out = out_buf[pad:pad + 3]
+    for num_splits in (0, 3):
+        assert mxa.mxa_device_error(True) == mxa.MXA_OK
+        _, lse = mxa.decode(inp.q.to(d), inp.k_cache.to(d), inp.v_cache.to(d), inp.block_table.to(d), sl.to(d),
+                            scale=w.scale, causal=False, max_seqlen_k=64, num_splits=num_splits, out=out)
+        torch.cuda.synchronize()
+        assert mxa.mxa_device_error(True) == mxa.MXA_ERR_INVALID_ARG
+        assert (out_buf[:pad] == 7).all() and (out_buf[pad + 3:] == 7).all()
+        ref_len = torch.tensor([40, min(max(bad_len, 0), 64), 33], dtype=torch.int32)
+        ro, rl = oracle.decode(inp.q, inp.k_cache, inp.v_cache, inp.block_table, ref_len, Hkv=2, page_size=16,
+                               dtype="bf16", scale=w.scale, causal=False)
+        assert_out_close(out.cpu(), ro, "bf16")
+        assert_lse_close(lse.cpu(), rl)
+
+
+def test_lengths_at_the_bounds_are_not_reported():
+    # 0 and max_seqlen_k themselves are valid lengths
+    w = Workload(name="edgelen", B=3, q_len=1, Hq=8, Hkv=2, D=128, dtype="bf16", page_size=16, causal=False,
+                 lengths="list:0,64,33", seed=547)
+    inp = make_inputs(w)
+    assert mxa.mxa_device_error(True) == mxa.MXA_OK
+    out, lse, _ = run_gpu(inp)
+    check(inp, out, lse)

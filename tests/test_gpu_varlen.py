@@ -98,7 +98,7 @@ def test_equal_counts_are_bit_identical_to_fixed_q_len(causal):
 def test_offsets_out_of_range_stay_in_bounds():
     # offsets that break the rules (past total_q, decreasing, a count above
     # max_seqlen_q) are clamped on the device: nothing outside out / lse is
-    # written, and the call completes
+    # written, the call completes, and the breach is reported
     c = CASES[0]
     w, inp, q, _ = draw(c, 780)
     total_q = q.shape[0]
@@ -113,7 +113,7 @@ def test_offsets_out_of_range_stay_in_bounds():
                       inp.cache_seqlens.to(d), max_seqlen_q=4, scale=w.scale, causal=True,
                       max_seqlen_k=inp.max_seqlen_k, out=out, lse=lse)
     torch.cuda.synchronize()
-    assert mxa.mxa_device_error(True) == mxa.MXA_OK
+    assert mxa.mxa_device_error(True) == mxa.MXA_ERR_INVALID_ARG
     assert (out_buf[:pad] == 7).all() and (out_buf[pad + total_q:] == 7).all()
     assert (lse_buf[:pad] == 7).all() and (lse_buf[pad + w.Hq * total_q:] == 7).all()
 

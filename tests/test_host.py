@@ -32,6 +32,24 @@ def test_library_exports_every_declared_symbol():
     assert sorted(mxa.EXPORTED) == names
 
 
+@pytest.mark.parametrize("splits", [1, 2, 3, 8, 16, 64])
+def test_workspace_size_is_the_uniform_plans(splits):
+    # the first phase of the two-phase call: the size mxa_plan puts in the
+    # plan, from the shape alone (no device for a uniform plan)
+    for p in (params(), params(B=5, q_len=4, Hq=32, Hkv=8, D=128, max_seqlen_k=8192, max_pages_per_seq=128),
+              params(B=3, q_len=1, Hq=16, Hkv=8, D=64, max_seqlen_k=300, max_pages_per_seq=19)):
+        plan = mxa.mxa_plan(p, splits, sm_count=148)
+        assert mxa.mxa_decode_workspace_size(p, splits) == plan.workspace_bytes
+        assert (plan.workspace_bytes > 0) == (splits > 1)
+
+
+def test_workspace_size_refusals():
+    assert mxa.mxa_decode_workspace_size(params(), -1) == mxa.SIZE_MAX
+    assert mxa.mxa_decode_workspace_size(params(D=96), 2) == mxa.SIZE_MAX
+    assert mxa.mxa_decode_workspace_size(params(Hq=30, Hkv=8), 2) == mxa.SIZE_MAX
+    assert mxa._lib.mxa_decode_workspace_size(None, 2) == mxa.SIZE_MAX
+
+
 def test_status_strings():
     for code in range(6):
         assert mxa.mxa_status_string(code).startswith("MXA_")
