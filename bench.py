@@ -76,6 +76,9 @@ def parse(argv=None):
     ap.add_argument("--varlen", action="store_true",
                     help="rows have their own query counts, drawn (seeded) from 1..q_len, packed with "
                          "cu_seqlens_q (mxa_decode_fwd_varlen)")
+    ap.add_argument("--combine", action="store_true",
+                    help="time the stand-alone merge (mxa_combine) of --num-splits float32 partial results of "
+                         "the workload's shape, instead of the decode")
     args = ap.parse_args(argv)
     if args.warmup < 0 or args.steps < 1:
         ap.error("--steps must be at least 1 and --warmup at least 0")
@@ -511,11 +514,48 @@ def e2e(r: Runner, case: Case, args):
                       "neighbouring steps' kernels"}
 
 
+def run_combine(args, r: Runner):
+    """The stand-alone merge of S float32 partial results (mxa_combine) for the
+    rows of the workload's shape: synthetic partials (N(0,1) rows, LSEs
+    N(0, 4^2) with some splits empty), W warm-up calls, then K timed calls.
+    Bytes per call: S partial rows and LSEs read, one output row and LSE
+    written per (b, t, h)."""
+    from decode_attention_packed_b200 import mxa
+    w = workload(args.workload)
+    S = args.num_splits or 16
+    g = torch.Generator(device="cpu").manual_seed(w.seed + 31)
+    rows = w.B * w.q_len * w.Hq
+    o = torch.randn((S, w.B, w.q_len, w.Hq, w.D), generator=g).to(r.dev)
+    lse_p = (torch.randn((S, w.B, w.Hq, w.q_len), generator=g) * 4).to(r.dev)
+    lse_p[S // 2] = float("-inf")  # an empty split
+    out = torch.empty((w.B, w.q_len, w.Hq, w.D), dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float16,
+                      device=r.dev)
+    lse = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=r.dev)
+    call = lambda i: mxa.mxa_combine(o, lse_p, out, lse, r.stream)  # noqa: E731
+    dev_s = r.timed(call, args.warmup, args.steps)
+    nbytes = S * rows * (w.D + 1) * 4 + rows * (w.D * out.element_size() + 4)
+    per = dev_s / args.steps
+    peak, peak_kind = measured_peak()
+    if r.rank == 0:
+        print(json.dumps({
+            "metric": "mxa_combine µs/call and GB/s (1 GPU)", "value": round(nbytes / per / 1e9, 2), "unit": "GB/s",
+            "n_gpus": r.world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per * 1e3, 5),
+            "us_per_call": round(per * 1e6, 3), "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "num_splits": S, "rows": rows, "D": w.D, "bytes_per_call": nbytes},
+            "roofline": {"bound": "hbm", "achieved": round(nbytes / per / 1e9, 2), "peak": peak, "unit": "GB/s",
+                         "frac": round(nbytes / per / 1e9 / peak, 4), "peak_kind": peak_kind,
+                         "kernel": "mxa_combine_kernel"},
+            "gpu_launches": args.steps}), flush=True)
+
+
 def main(argv=None):
     args = parse(argv)
     world, rank, local = setup_dist(args)
     if args.impl == "reference":
         run_reference(args, world, rank)
+        return
+    if args.combine:
+        run_combine(args, Runner(world, rank, local))
         return
 
     r = Runner(world, rank, local)

@@ -24,7 +24,7 @@ mxa_status_t check_shape(const mxa_decode_params_t *p) {
   if (p->dtype != MXA_F16 && p->dtype != MXA_BF16) return MXA_ERR_INVALID_ARG;
   if (p->page_size < 1 || p->num_pages < 1 || p->max_seqlen_k < 0 || p->max_pages_per_seq < 1)
     return MXA_ERR_INVALID_ARG;
-  if (p->D != 64 && p->D != 128) return MXA_ERR_UNSUPPORTED;
+  if (p->D != 64 && p->D != 128 && p->D != 256) return MXA_ERR_UNSUPPORTED;
   const long long T = block_tokens(p->D);
   const long long G = p->Hq / p->Hkv;
   const long long RT = ceil_div_ll((long long)p->q_len * G, kRowsPerTile);
@@ -125,7 +125,7 @@ const char *mxa_status_string(mxa_status_t s) {
   switch (s) {
     case MXA_OK: return "MXA_OK";
     case MXA_ERR_INVALID_ARG: return "MXA_ERR_INVALID_ARG: null or misaligned pointer, or inconsistent shape";
-    case MXA_ERR_UNSUPPORTED: return "MXA_ERR_UNSUPPORTED: shape not implemented (D must be 64 or 128; page size must tile the gather)";
+    case MXA_ERR_UNSUPPORTED: return "MXA_ERR_UNSUPPORTED: shape not implemented (D must be 64, 128 or 256; page size must tile the gather)";
     case MXA_ERR_WORKSPACE: return "MXA_ERR_WORKSPACE: workspace missing or smaller than the plan needs";
     case MXA_ERR_CUDA: return "MXA_ERR_CUDA: a CUDA runtime call failed";
     case MXA_ERR_TIMEOUT: return "MXA_ERR_TIMEOUT: a device-side bounded wait ran out";

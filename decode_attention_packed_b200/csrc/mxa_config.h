@@ -38,12 +38,16 @@ constexpr int kErrInputMask = kErrBadPage | kErrBadLen | kErrBadOffsets;
 // packed query rows, and measures at about one block per two rows on B200.
 constexpr int unit_cost_for_rows(int rows) { return rows > 2 ? (rows + 1) / 2 : 1; }
 
-// KV tokens per pipeline stage: every stage carries T x D elements of K and
-// of V (16 KiB each in 16-bit types), so T = 8192 / D.  Three stages per CTA
-// and two CTAs per SM keep 192 KiB of loads in flight per SM, which is what
-// B200's HBM needs at its loaded latency of several microseconds; two CTAs
-// also let one stream while the other starts up or finishes.
-constexpr int block_tokens(int D) { return 8192 / D; }
+// KV tokens per pipeline stage.  For D <= 128 every stage carries T x D
+// elements of K and of V (16 KiB each in 16-bit types), so T = 8192 / D:
+// three stages per CTA and two CTAs per SM keep 192 KiB of loads in flight
+// per SM, which is what B200's HBM needs at its loaded latency of several
+// microseconds; two CTAs also let one stream while the other starts up or
+// finishes.  For D = 256 a stage is 64 keys (32 KiB of K and of V) and one
+// CTA holds an SM: the same 192 KiB in flight, and the math warps keep the
+// whole 256-column accumulator in registers (one CTA per SM leaves them 255
+// registers a thread), each on 16 keys of a stage as for D = 128.
+constexpr int block_tokens(int D) { return D <= 128 ? 8192 / D : 64; }
 
 constexpr size_t stage_bytes(int D) { return (size_t)2 * block_tokens(D) * D * 2; }
 constexpr int q_row_pitch(int D) { return D * 2; }
@@ -87,12 +91,12 @@ constexpr size_t smem_jobs_off(int D) { return smem_desc_off(D) + sizeof(Segment
 // The epilogue warp's staging buffer, used in turn for the rows of a job's
 // output before their bulk (TMA) stores (up to 16 rows x D fp32), and as the
 // landing zone of the pieces of a split unit being merged (partial rows
-// first, then the 16 LSE values of each piece).
-constexpr size_t kLandRows = 8 * 1024;
-constexpr size_t kLandBytes = kLandRows + 16 * kRowsPerTile * 4;
-constexpr size_t out_stage_bytes(int D) {
-  return (size_t)kRowsPerTile * D * 4 > kLandBytes ? (size_t)kRowsPerTile * D * 4 : kLandBytes;
+// first, at least one whole 16-row piece, then the 16 row values of each of
+// up to 16 pieces).
+constexpr size_t land_rows_bytes(int D) {
+  return (size_t)kRowsPerTile * D * 4 > 8 * 1024 ? (size_t)kRowsPerTile * D * 4 : 8 * 1024;
 }
+constexpr size_t out_stage_bytes(int D) { return land_rows_bytes(D) + 16 * kRowsPerTile * 4; }
 constexpr size_t smem_out_off(int D) { return smem_jobs_off(D) + kJobs * sizeof(JobSlot); }
 constexpr size_t smem_bar_off(int D) { return smem_out_off(D) + out_stage_bytes(D); }
 constexpr size_t smem_total(int D) { return smem_bar_off(D) + kBarrierBytes; }
@@ -119,6 +123,9 @@ static_assert(2 * (smem_total(128) + kSmemReservedPerCta) <= (size_t)kSmemPerSm,
               "D = 128 layout must leave room for two CTAs per SM");
 static_assert(2 * (smem_total(64) + kSmemReservedPerCta) <= (size_t)kSmemPerSm,
               "D = 64 layout must leave room for two CTAs per SM");
+static_assert(smem_total(256) + kSmemReservedPerCta <= (size_t)kSmemPerSm && smem_total(256) <= 227 * 1024,
+              "D = 256 layout must fit one CTA per SM");
+static_assert(ctas_per_sm(64) == 2 && ctas_per_sm(128) == 2 && ctas_per_sm(256) == 1, "CTAs per SM");
 static_assert((size_t)kMaxBalancedRows * 8 <= kStages * stage_bytes(64), "prologue scan fits the ring");
 
 }  // namespace mxa

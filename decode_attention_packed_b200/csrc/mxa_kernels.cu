@@ -660,6 +660,14 @@ __device__ void math_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lan
       if (r >= rows) qa[kk][0] = qa[kk][2] = 0u;
       if (r + 8 >= rows) qa[kk][1] = qa[kk][3] = 0u;
     }
+    // The Q tile is refilled by the next segment's bulk copies (the async
+    // proxy) as soon as every math warp has arrived below.  These fragments
+    // are first used by the block loop's tensor-core instructions, after the
+    // arrival, so without a proxy fence the last ldmatrix reads may still be
+    // in flight when the copies land: the high columns of a row then come
+    // from the next segment's queries.  The fence orders this warp's reads
+    // before the refill.
+    fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(qempty);
     ++seg_k;
@@ -856,7 +864,10 @@ __device__ void math_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lan
 template <int D>
 __device__ __forceinline__ void stage_f32_vec(uint8_t *smem, uint32_t stage, int rr, int col, const float *v) {
   float *dst = reinterpret_cast<float *>(smem + (stage - smem_addr(smem))) + rr * D + col;
-  if constexpr (D / 32 == 4) {
+  if constexpr (D / 32 == 8) {
+    reinterpret_cast<float4 *>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4 *>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else if constexpr (D / 32 == 4) {
     *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
   } else {
     *reinterpret_cast<float2 *>(dst) = make_float2(v[0], v[1]);
@@ -869,7 +880,10 @@ __device__ __forceinline__ void stage_f32_vec(uint8_t *smem, uint32_t stage, int
 template <int D, bool kBf16>
 __device__ __forceinline__ void stage_out_vec(uint8_t *smem, uint32_t stage, int rr, int col, const float *v) {
   uint8_t *dst = smem + (stage - smem_addr(smem)) + (rr * D + col) * 2;
-  if constexpr (D / 32 == 4) {
+  if constexpr (D / 32 == 8) {
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(pack2<kBf16>(v[0], v[1]), pack2<kBf16>(v[2], v[3]),
+                                                 pack2<kBf16>(v[4], v[5]), pack2<kBf16>(v[6], v[7]));
+  } else if constexpr (D / 32 == 4) {
     *reinterpret_cast<uint2 *>(dst) = make_uint2(pack2<kBf16>(v[0], v[1]), pack2<kBf16>(v[2], v[3]));
   } else {
     *reinterpret_cast<uint32_t *>(dst) = pack2<kBf16>(v[0], v[1]);
@@ -1077,7 +1091,12 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
           const float l = lp[rr] * kLog2e;
           w = l == -INFINITY ? 0.f : ex2(l - row_lse[rr]);
         }
-        if constexpr (VEC == 4) {
+        if constexpr (VEC == 8) {
+          const float4 v = reinterpret_cast<const float4 *>(op + rc * D)[0];
+          const float4 u = reinterpret_cast<const float4 *>(op + rc * D)[1];
+          acc[rr][0] += w * v.x; acc[rr][1] += w * v.y; acc[rr][2] += w * v.z; acc[rr][3] += w * v.w;
+          acc[rr][4] += w * u.x; acc[rr][5] += w * u.y; acc[rr][6] += w * u.z; acc[rr][7] += w * u.w;
+        } else if constexpr (VEC == 4) {
           const float4 v = *reinterpret_cast<const float4 *>(op + rc * D);
           acc[rr][0] += w * v.x; acc[rr][1] += w * v.y; acc[rr][2] += w * v.z; acc[rr][3] += w * v.w;
         } else {
@@ -1244,7 +1263,7 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
     const uint32_t pbytes = (uint32_t)rows * D * 4;
     const int own = (int)blockIdx.x - sg.c_first;  // this piece's index in the unit
     bool hold = false, merge_now = false;
-    uint32_t land = oland, land_rows = (uint32_t)kLandRows, dst_rows = ostage;
+    uint32_t land = oland, land_rows = (uint32_t)land_rows_bytes(D), dst_rows = ostage;
     int lse_slots = kRowsPerTile;
     auto merge_warps = [&](auto row_slots) {
       constexpr int NR = decltype(row_slots)::value;
@@ -1258,7 +1277,13 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
         for (int w = 0; w < kMathWarps; ++w) {
           const float wg = __shfl_sync(0xffffffffu, wgt[w], rr);
           const float *src = hbase + (handoff_addr<D>(sbase, w, rc, col) - sbase) / 4;
-          if constexpr (VEC == 4) {
+          if constexpr (VEC == 8) {  // two 16-byte chunks, each at its own swizzled place
+            const float4 v = *reinterpret_cast<const float4 *>(src);
+            const float4 u =
+                *reinterpret_cast<const float4 *>(hbase + (handoff_addr<D>(sbase, w, rc, col + 4) - sbase) / 4);
+            acc[rr][0] += wg * v.x; acc[rr][1] += wg * v.y; acc[rr][2] += wg * v.z; acc[rr][3] += wg * v.w;
+            acc[rr][4] += wg * u.x; acc[rr][5] += wg * u.y; acc[rr][6] += wg * u.z; acc[rr][7] += wg * u.w;
+          } else if constexpr (VEC == 4) {
             const float4 v = *reinterpret_cast<const float4 *>(src);
             acc[rr][0] += wg * v.x; acc[rr][1] += wg * v.y; acc[rr][2] += wg * v.z; acc[rr][3] += wg * v.w;
           } else {
@@ -1270,11 +1295,11 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
       seen = __shfl_sync(0xffffffffu, seen, 0);
       const bool all_here = sg.kind != 0 && (seen >> 32) == (unsigned long long)a.epoch &&
                             (int)(seen & 0xffffffffull) == sg.n_pieces - 1;
-      hold = all_here && !sg.last && (uint32_t)sg.n_pieces * pbytes > (uint32_t)kLandRows &&
+      hold = all_here && !sg.last && (uint32_t)sg.n_pieces * pbytes > (uint32_t)land_rows_bytes(D) &&
              sg.n_pieces <= min(kRowsPerTile, (int)(stage_land_rows<D>() / pbytes));
       land = sg.last ? ring : hold ? sbase : oland;
       land_rows = sg.last ? kStages * 2 * KV_BYTES - kRingLseSlots * kRowsPerTile * 4
-                  : hold ? stage_land_rows<D>() : (uint32_t)kLandRows;
+                  : hold ? stage_land_rows<D>() : (uint32_t)land_rows_bytes(D);
       lse_slots = sg.last ? kRingLseSlots : kRowsPerTile;
       merge_now = all_here && sg.n_pieces <= min(lse_slots, (int)(land_rows / pbytes));
       __syncwarp();  // every lane has read the stage before it may become the landing zone
@@ -1360,7 +1385,7 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
 // The split kernel
 // ---------------------------------------------------------------------------
 template <int D, bool kBf16, bool kAppend, bool kVarlen>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, ctas_per_sm(D))
     mxa_split_kernel(const __grid_constant__ TmapPair tm, const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1625,6 +1650,7 @@ mxa_status_t launch_decode(const DecodeLaunch &L, cudaStream_t stream) {
   const bool bf16 = L.p.dtype == MXA_BF16;
   if (L.p.D == 128) return bf16 ? launch_typed<128, true>(L, stream) : launch_typed<128, false>(L, stream);
   if (L.p.D == 64) return bf16 ? launch_typed<64, true>(L, stream) : launch_typed<64, false>(L, stream);
+  if (L.p.D == 256) return bf16 ? launch_typed<256, true>(L, stream) : launch_typed<256, false>(L, stream);
   return MXA_ERR_UNSUPPORTED;
 }
 

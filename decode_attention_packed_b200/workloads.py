@@ -78,10 +78,15 @@ WORKLOADS = [
 
 # Other readings of the workloads above, benchmarked for context only: the
 # speculative step with every row at 8192 keys (the spec/MTP lengths read as
-# "all rows 8192" instead of the cycle through the non-power-of-two lengths).
+# "all rows 8192" instead of the cycle through the non-power-of-two lengths);
+# and head dim 256, the wider head a model family of the MXFlashAttn page
+# uses (its split-KV kernel hands that shape back to a fallback path), as a
+# GQA decode batch: groups of 4, 16-slot pages in a seeded permutation.
 CONTEXT_WORKLOADS = [
     Workload("spec_mtp_small_q_all8192", B=16, q_len=4, Hq=32, Hkv=8, D=128, dtype="bf16",
              page_size=64, causal=True, lengths="const:8192", seed=1012),
+    Workload("gqa_decode_hd256", B=32, q_len=1, Hq=16, Hkv=4, D=256, dtype="bf16",
+             page_size=16, causal=False, lengths="uniform:1:4096", seed=1013),
 ]
 
 BY_NAME = {w.name: w for w in WORKLOADS + CONTEXT_WORKLOADS}

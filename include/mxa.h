@@ -10,7 +10,8 @@
  * O = softmax(Q K^T / sqrt(headDim)) V with small qLen and long kvLen), on the
  * paged KV cache of the "MXFlashAttn 1.4.0" project page (能力矩阵, the
  * capability matrix: paged KV cache, FP16/BF16 forward, head_dim 64/128,
- * GQA), computed with the online softmax of the "ops-transformer
+ * GQA; head_dim 256, which the same page's split-KV kernel hands back to a
+ * fallback path, is served here by the same kernel), computed with the online softmax of the "ops-transformer
  * FlashAttention" walkthrough (section "FlashAttention 的数学细节"), the
  * query-head packing and KV-axis split of "Flash-Attention GQA 性能调优:
  * pack_gqa 与 num_splits 两个开关怎么选" (section "两个开关在 kernel 层面各做
@@ -52,7 +53,7 @@ extern "C" {
 typedef enum {
   MXA_OK = 0,
   MXA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad shape or stride */
-  MXA_ERR_UNSUPPORTED = 2,   /* a shape the kernels do not implement (e.g. D not 64/128) */
+  MXA_ERR_UNSUPPORTED = 2,   /* a shape the kernels do not implement (e.g. D not 64/128/256) */
   MXA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than mxa_plan() says */
   MXA_ERR_CUDA = 4,          /* a CUDA runtime call failed (no device, launch error) */
   MXA_ERR_TIMEOUT = 5        /* a device-side bounded wait ran out (see mxa_device_error) */
@@ -112,8 +113,8 @@ typedef struct {
   int grid;              /* CTAs of the split kernel */
   int units;             /* B * Hkv * ceil(q_len * G / 16) */
   int rows_per_tile;     /* packed query rows per tile (16) */
-  int block_tokens;      /* KV tokens per pipeline stage */
-  int ctas_per_sm;       /* resident CTAs per SM the plan assumed */
+  int block_tokens;      /* KV tokens per pipeline stage: 8192 / D for D <= 128, 64 for D = 256 */
+  int ctas_per_sm;       /* resident CTAs per SM the plan assumed: 2, or 1 for D = 256 */
   int sm_count;          /* SMs the plan assumed */
   int needs_combine;     /* 1 if units may be split across CTAs and merged (needs the workspace) */
   int unit_cost;         /* BALANCED: fixed cost of a unit, in KV blocks, added to its blocks
@@ -163,7 +164,7 @@ MXA_API int mxa_num_splits_heuristic(int tiles, int sm_count, int slots, int num
  *   sm_count <= 0  : query the current CUDA device (MXA_ERR_CUDA without one).
  * Errors: MXA_ERR_INVALID_ARG for a NULL pointer or an inconsistent shape
  * (B < 0, q_len < 1, Hq % Hkv != 0, page_size < 1, ...);
- * MXA_ERR_UNSUPPORTED for D not in {64, 128} or sizes past the int32
+ * MXA_ERR_UNSUPPORTED for D not in {64, 128, 256} or sizes past the int32
  * index range.  The page size is checked by the run calls, which know
  * whether the cache is paged: a paged cache needs page_size to divide the
  * stage of block_tokens tokens and be a multiple of 8, or to be a multiple

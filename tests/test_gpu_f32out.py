@@ -100,7 +100,8 @@ def test_ragged_balanced_grids_raw(grid):
 EDGE = [0, 1, 2, 15, 16, 17, 63, 64, 65, 127, 128, 129, 255, 257, 1023, 1025, 1500, 3000, 4096]
 
 
-@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f16", 64), ("bf16", 64), ("f16", 128)])
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f16", 64), ("bf16", 64), ("f16", 128), ("bf16", 256),
+                                     ("f16", 256)])
 def test_edge_lengths_raw(dtype, D):
     w = Workload(name="edge32", B=len(EDGE), q_len=1, Hq=8, Hkv=2, D=D, dtype=dtype, page_size=16,
                  causal=False, lengths="list:" + ",".join(map(str, EDGE)), seed=31)
@@ -129,3 +130,47 @@ def test_f32out_refuses_bad_arguments():
     p.D = 128
     st = mxa._lib.mxa_decode_fwd_f32out(None, None, None, None, None, p, 0.1, 0, None, None, 0, None, None, None)
     assert st == mxa.MXA_ERR_INVALID_ARG
+
+
+def test_head_dim_256_full_size_raw():
+    from decode_attention_packed_b200.workloads import workload
+    inp = make_inputs(workload("gqa_decode_hd256"))
+    err, plan = check(inp)
+    print(f"gqa_decode_hd256: raw max|err| (float32 O) = {err:.3e}, plan grid {plan.grid}")
+
+
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f16", 64)])
+def test_two_cache_segments_merge_through_combine(dtype, D):
+    # Each row's keys are cut at a page boundary into two segments; each
+    # segment is decoded on its own with a float32 output and its LSE, and
+    # mxa_combine merges the two partial results into the decode of the
+    # whole cache (the use the float32 output is offered for).
+    w = Workload(name="segments", B=6, q_len=1, Hq=16, Hkv=4, D=D, dtype=dtype, page_size=16, causal=False,
+                 lengths="list:1,31,40,300,1025,2048", seed=77)
+    inp = make_inputs(w)
+    ro, rl = oracle_of(inp)
+    L = inp.cache_seqlens.numpy()
+    bt = inp.block_table.numpy()
+    first_pages = [(int(x) // 16) // 2 for x in L]  # segment A: the first half of the full pages
+    la_len = np.array([p * 16 for p in first_pages], dtype=np.int32)
+    lb_len = (L - la_len).astype(np.int32)
+    bt_b = np.zeros_like(bt)
+    for b, p in enumerate(first_pages):
+        bt_b[b, :bt.shape[1] - p] = bt[b, p:]
+    d = "cuda"
+    q, k, v = inp.q.to(d), inp.k_cache.to(d), inp.v_cache.to(d)
+    parts = []
+    for table, lens in ((bt, la_len), (bt_b, lb_len)):
+        o, l = mxa.decode(q, k, v, torch.from_numpy(table).to(d), torch.from_numpy(lens).to(d), scale=w.scale,
+                          causal=False, max_seqlen_k=inp.max_seqlen_k, out_dtype=torch.float32)
+        parts.append((o, l))
+    o_part = torch.stack([parts[0][0], parts[1][0]])  # [2, B, q_len, Hq, D]
+    lse_part = torch.stack([parts[0][1], parts[1][1]])  # [2, B, Hq, q_len]
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=d)
+    mxa.mxa_combine(o_part, lse_part, out, lse)
+    torch.cuda.synchronize()
+    assert mxa.mxa_device_error(True) == mxa.MXA_OK
+    from tests.tolerance import assert_out_close
+    assert_out_close(out.cpu(), ro, dtype)
+    assert_lse_close(lse.cpu(), rl)

@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import oracle
-from decode_attention_packed_b200.workloads import WORKLOADS, Workload, make_inputs
+from decode_attention_packed_b200.workloads import WORKLOADS, Workload, make_inputs, workload
 from tests.tolerance import assert_lse_close, assert_out_close
 
 pytestmark = pytest.mark.gpu
@@ -176,7 +176,7 @@ def wl(**kw):
     return Workload(**base)
 
 
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("num_splits", [0, 1, 3])
 def test_edge_lengths(D, dtype, num_splits):
@@ -187,7 +187,7 @@ def test_edge_lengths(D, dtype, num_splits):
 
 
 @pytest.mark.parametrize("page", [0, 8, 16, 32, 64, 128, 256, 192])
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D", [64, 128, 256])
 def test_page_sizes(page, D):
     if page == 192 and D == 64:
         pytest.skip("192 neither divides nor is a multiple of the 128-key stage of D = 64")
@@ -373,3 +373,71 @@ def test_lengths_at_the_bounds_are_not_reported():
     assert mxa.mxa_device_error(True) == mxa.MXA_OK
     out, lse, _ = run_gpu(inp)
     check(inp, out, lse)
+
+
+
+# --------------------------------------------------------------------------
+# head dim 256: 64-key stages of 64 KiB, one CTA per SM
+# --------------------------------------------------------------------------
+
+def test_head_dim_256_full_size():
+    inp = make_inputs(workload("gqa_decode_hd256"))
+    ref = run_oracle(inp)
+    for s in (0, 1, 4):
+        out, lse, plan = run_gpu(inp, num_splits=s)
+        assert plan.ctas_per_sm == 1 and plan.block_tokens == 64
+        err = check(inp, out, lse, ref)
+        print(f"gqa_decode_hd256 splits={s}: grid {plan.grid} max|err|={err:.3e}")
+
+
+@pytest.mark.parametrize("G,q_len,causal", [(1, 1, False), (2, 4, True), (4, 4, True), (8, 2, False),
+                                            (16, 1, False), (4, 8, True)])
+def test_head_dim_256_groups_and_query_lengths(G, q_len, causal):
+    inp = make_inputs(wl(Hq=2 * G, Hkv=2, q_len=q_len, causal=causal, D=256, lengths="list:1,9,130,1025,3000",
+                         B=5, page_size=32, seed=600 + G * 10 + q_len))
+    for s in (0, 2):
+        out, lse, _ = run_gpu(inp, num_splits=s)
+        check(inp, out, lse)
+
+
+@pytest.mark.parametrize("grid", [1, 7, 148, 1000])
+def test_head_dim_256_balanced_grids(grid):
+    inp = make_inputs(wl(D=256, lengths="uniform:0:3000", B=24, Hq=16, Hkv=4, page_size=64, seed=640))
+    q, k, v, bt, sl = to_dev(inp)
+    plan = mxa.mxa_plan_balanced(mxa.params_for(q, k, bt, inp.max_seqlen_k), grid)
+    out, lse, _ = run_gpu(inp, plan=plan, dev=(q, k, v, bt, sl))
+    check(inp, out, lse)
+
+
+# --------------------------------------------------------------------------
+# repeated calls on a garbage workspace
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name,grid", [("ragged_varlen", 296), ("gqa_decode", 296), ("spec_mtp_small_q", 296),
+                                       ("gqa_decode_hd256", 148)])
+def test_repeated_calls_on_a_garbage_workspace(name, grid):
+    # 200 calls in a row, each on a workspace whose every byte is 0xFF (NaN
+    # partial results, all-ones arrival counters): every call must match the
+    # oracle.  A read of a partial result before it is written shows up as
+    # NaN; a read of a shared-memory tile while it is being refilled for the
+    # next segment shows up as a wrong row in a few calls out of a hundred.
+    w = workload(name)
+    inp = make_inputs(w)
+    ro, _ = run_oracle(inp)
+    q, k, v, bt, sl = to_dev(inp)
+    params = mxa.params_for(q, k, bt, inp.max_seqlen_k)
+    plan = mxa.mxa_plan_balanced(params, grid)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    lse = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device="cuda")
+    ref = torch.from_numpy(ro).cuda()
+    worst = torch.zeros((), dtype=torch.float64, device="cuda")
+    for _ in range(200):
+        ws.fill_(255)
+        out.fill_(float("nan"))
+        mxa.mxa_decode_fwd_f32out(q, k, v, bt, sl, params, w.scale, w.causal, plan, ws, out, lse)
+        err = torch.nan_to_num((out.double() - ref).abs(), nan=1e9).max()
+        worst = torch.maximum(worst, err)
+    torch.cuda.synchronize()
+    assert mxa.mxa_device_error(True) == mxa.MXA_OK
+    assert worst.item() <= 2e-3, f"worst |err| over 200 calls: {worst.item():.3e}"

@@ -3,8 +3,9 @@
 The queries are packed as q [total_q, Hq, D] with offsets cu_seqlens_q
 [B + 1]; the oracle's decode_varlen is the reference.  The cases mix rows
 without queries, rows without keys, rows whose causal queries see no key,
-one and two row tiles per KV head, both schedules, D = 64 and 128, fp16 and
-bf16, paged and contiguous caches.
+one and two row tiles per KV head, both schedules, D = 64, 128 and 256, fp16
+and bf16, paged and contiguous caches, and a full-size speculative batch with
+counts drawn from {0, 1, 2, 4, 8}.
 """
 import numpy as np
 import pytest
@@ -39,6 +40,12 @@ CASES = [
     # rows with queries but no keys, and with keys but no queries
     dict(q_lens=[3, 0, 2, 1], Hq=8, Hkv=2, D=128, dtype="bf16", page_size=16, causal=True,
          lengths=[0, 50, 0, 900]),
+    # head dim 256, counts 0..8: a row of 8 queries in groups of 4 spans two row tiles
+    dict(q_lens=[8, 1, 4, 0, 2], Hq=16, Hkv=4, D=256, dtype="bf16", page_size=32, causal=True,
+         lengths=[9, 700, 2049, 40, 3000]),
+    # counts 8 in groups of 2: exactly one full 16-row tile
+    dict(q_lens=[8, 8, 1, 0], Hq=8, Hkv=4, D=64, dtype="f16", page_size=16, causal=False,
+         lengths=[8, 513, 4096, 77]),
 ]
 
 
@@ -74,6 +81,23 @@ def test_varlen_matches_oracle(case, num_splits):
                                   causal=c["causal"])
     assert_out_close(out, ro, w.dtype)
     assert_lse_close(lse, rl)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_full_size_speculative_batch_with_mixed_counts(causal):
+    # the speculative workload's shape (16 rows, 32 query heads in groups of
+    # 4, head dim 128, bf16, pages of 64, lengths 8192 / 1023 / 1025 / 1500 /
+    # 3000) with per-row query counts drawn from {0, 1, 2, 4, 8}
+    lengths = [[8192, 1023, 1025, 1500, 3000][b % 5] for b in range(16)]
+    q_lens = np.random.default_rng(811).choice([0, 1, 2, 4, 8], size=16).tolist()
+    c = dict(q_lens=q_lens, Hq=32, Hkv=8, D=128, dtype="bf16", page_size=64, causal=causal, lengths=lengths)
+    w, inp, q, cu = draw(c, 810 + int(causal))
+    ro, rl = oracle.decode_varlen(q, cu.numpy(), inp.k_cache, inp.v_cache, inp.block_table, inp.cache_seqlens,
+                                  Hkv=w.Hkv, page_size=inp.page_size, dtype=w.dtype, scale=w.scale, causal=causal)
+    for num_splits in (0, 4):
+        out, lse = run_varlen(inp, q, cu, 8, causal, num_splits)
+        assert_out_close(out, ro, w.dtype)
+        assert_lse_close(lse, rl)
 
 
 @pytest.mark.parametrize("causal", [False, True])

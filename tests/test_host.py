@@ -164,7 +164,8 @@ def test_plan_switches_to_uniform_past_the_balanced_row_limit():
 
 @pytest.mark.parametrize("kw,code", [
     (dict(D=96), MXA_ERR_UNSUPPORTED),
-    (dict(D=256), MXA_ERR_UNSUPPORTED),
+    (dict(D=512), MXA_ERR_UNSUPPORTED),
+    (dict(D=192), MXA_ERR_UNSUPPORTED),
     (dict(Hq=12, Hkv=8), MXA_ERR_INVALID_ARG),
     (dict(q_len=0), MXA_ERR_INVALID_ARG),
     (dict(B=-1), MXA_ERR_INVALID_ARG),
@@ -175,6 +176,22 @@ def test_plan_refuses_bad_shapes(kw, code):
     plan = mxa_plan_t()
     p = params(**kw)
     assert mxa._lib.mxa_plan(ctypes.byref(p), 0, 148, ctypes.byref(plan)) == code
+
+
+def test_plan_head_dim_256_holds_one_cta_per_sm():
+    # 64-key stages of 64 KiB, three in the ring: one CTA per SM, so the
+    # automatic plan's full wave is one CTA per SM
+    p = params(D=256, B=32, Hq=16, Hkv=4, max_seqlen_k=4096, max_pages_per_seq=256, num_pages=8192, page_size=16)
+    plan = mxa.mxa_plan(p, 0, sm_count=148)
+    assert plan.ctas_per_sm == 1 and plan.block_tokens == 64
+    assert plan.schedule == MXA_SCHED_BALANCED and plan.grid == 148
+    for D, cps, T in ((64, 2, 128), (128, 2, 64)):
+        q = mxa.mxa_plan(params(D=D), 0, sm_count=148)
+        assert (q.ctas_per_sm, q.block_tokens) == (cps, T)
+    # a 16-row piece of head dim 256 is 16 KiB in float32: the workspace holds
+    # two such slots per CTA after the counters
+    u = mxa.mxa_plan(p, 3, sm_count=148)
+    assert u.workspace_bytes >= u.grid * 2 * 16 * 256 * 4
 
 
 def _run_with_plan(p, plan, *, q=1, k=1, v=1, bt=1, sl=1, out=1, ws=None, ws_bytes=0, lse=None,
