@@ -468,11 +468,10 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
     if constexpr (kAppend) new0 = a.seqlens[seg.b];
     Window win;
     load_window(seg, win);
-    if (!warp_wait_bounded(qempty, 1, &g_mxa_err, kErrWaitQ, lane)) ok = false;  // first use: free
-    if (ok) {
-      issue_q(seg);
-      ++seg_k;
-    }
+    // The first segment's Q rows are requested after its first KV stage:
+    // the TMA unit serves copies in turn, and the KV bytes have the longer
+    // way to come.  The Q slot is free on first use.
+    bool q_first = true;
     while (ok) {
       bool have_next = false, next_known = false, q_next = false;
       SegmentDesc nseg;
@@ -535,6 +534,11 @@ __device__ void producer_warp(const TmapPair &tm, const DecodeArgs &a, uint8_t *
           }
         }
         ++it;
+        if (q_first) {
+          q_first = false;
+          issue_q(seg);
+          ++seg_k;
+        }
         // Find the next segment once this one's first stage is on its way
         // (its loads then hide behind this segment's stages).
         if (!next_known) {
