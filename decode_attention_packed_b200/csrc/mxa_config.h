@@ -77,10 +77,10 @@ struct JobSlot {
   float ml[kMathWarps][kRowsPerTile][2];
 };
 
-// full[S], empty[S], qfull, qempty, job_full[J], job_empty[J], merge, init;
-// then the two split units whose counters the CTA tags (2 ints)
+// full[S], empty[S], qfull, qempty, job_full[J], job_empty[J], merge, init,
+// final; then the two split units whose counters the CTA tags (2 ints)
 constexpr size_t kBarrierBytes = 128;
-constexpr int kNumBarriers = 2 * kStages + 2 + 2 * kJobs + 2;
+constexpr int kNumBarriers = 2 * kStages + 2 + 2 * kJobs + 3;
 constexpr size_t kInitUnitsOff = (size_t)kNumBarriers * 8;
 
 // Offsets inside the dynamic shared memory (base aligned to 1024 bytes).
@@ -98,7 +98,10 @@ constexpr size_t land_rows_bytes(int D) {
 }
 constexpr size_t out_stage_bytes(int D) { return land_rows_bytes(D) + 16 * kRowsPerTile * 4; }
 constexpr size_t smem_out_off(int D) { return smem_jobs_off(D) + kJobs * sizeof(JobSlot); }
-constexpr size_t smem_bar_off(int D) { return smem_out_off(D) + out_stage_bytes(D); }
+// The epilogue warp's note to the math warps about the CTA's final merge.
+constexpr size_t kFinalBytes = 128;
+constexpr size_t smem_final_off(int D) { return smem_out_off(D) + out_stage_bytes(D); }
+constexpr size_t smem_bar_off(int D) { return smem_final_off(D) + kFinalBytes; }
 constexpr size_t smem_total(int D) { return smem_bar_off(D) + kBarrierBytes; }
 
 constexpr int ctas_per_sm(int D) {

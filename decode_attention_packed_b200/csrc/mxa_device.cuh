@@ -142,6 +142,22 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+__device__ __forceinline__ bool warp_wait_bounded_idle(uint32_t bar, uint32_t parity, int *err_flag,
+                                                       int code, int lane) {
+  bool mine = mbar_try_wait(bar, parity);
+  if (__all_sync(0xffffffffu, mine)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(128);
+    if (!mine) mine = mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, mine)) return true;
+    if ((i & 63u) == 0 && __any_sync(0xffffffffu, globaltimer_ns() - t0 > kWaitLimitNs)) {
+      if (lane == 0) atomicOr(err_flag, code);
+      return false;
+    }
+  }
+}
+
 // 3-D tiled TMA load global -> shared, completing on `bar` (tx bytes), with
 // an L2 cache policy (from l2_policy_evict_first).
 __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const void *tmap, int x, int y, int z,

@@ -62,7 +62,60 @@ constexpr int B_JOBFULL(int j) { return 2 * kStages + 2 + j; }
 constexpr int B_JOBEMPTY(int j) { return 2 * kStages + 2 + kJobs + j; }
 constexpr int B_MERGE = 2 * kStages + 2 + 2 * kJobs;  // pieces of a split unit landed by bulk loads
 constexpr int B_INIT = B_MERGE + 1;                     // the producer has published the CTA's split units
+constexpr int B_FINAL = B_INIT + 1;                     // the epilogue warp has posted the CTA's final merge
 constexpr int kRingLseSlots = 32;                       // pieces' LSEs a merge landing in the ring holds
+
+// Posted by the epilogue warp at the end of the CTA's work: whether the
+// math warps join the second pass of the merge of the unit of the CTA's last
+// job, and where its pieces have landed.
+struct FinalMerge {
+  SegmentDesc seg;
+  int valid;                   // 1: join the merge
+  int rows;                    // packed rows of the unit
+  uint32_t land, land_rows;    // landing zone (shared-memory address) and its bytes of rows
+  float lse2[kRowsPerTile];    // the rows' LSEs, base 2
+};
+static_assert(sizeof(FinalMerge) <= kFinalBytes, "the final merge's record fits its slot");
+
+// Second pass of the merge of the CTA's final split unit, shared by the
+// epilogue warp and the math warps (warp `wid` of kMathWarps + 1) once the
+// epilogue warp has landed every piece and found the rows' LSEs:
+// O = sum_i w_i O_i with w_i = exp(lse_i - LSE), one (row, 4 columns) item
+// at a time, straight to the output.  The terms and their order are those of
+// merge_pieces' own second pass, so a unit's result does not depend on which
+// path merged it.
+template <int D, bool kBf16>
+__device__ void merge_pass2_coop(const DecodeArgs &a, const FinalMerge *fm, const uint8_t *smem, int wid,
+                                 int lane) {
+  constexpr int CW = D / 4;  // 4-column items of a row
+  constexpr float kLog2e = 1.4426950408889634f;
+  const int rows = fm->rows, n = fm->seg.n_pieces;
+  const int rt = fm->seg.rt, h = fm->seg.h, q0 = fm->seg.q0;
+  const uint32_t sbase = smem_addr(smem);
+  const float *land_o = reinterpret_cast<const float *>(smem + (fm->land - sbase));
+  const float *land_l = reinterpret_cast<const float *>(smem + (fm->land + fm->land_rows - sbase));
+  // the epilogue warp, which posted the pass and is awake, takes the first items
+  const int first = (wid == kMathWarps ? 0 : wid + 1) * 32 + lane;
+  for (int item = first; item < rows * CW; item += (kMathWarps + 1) * 32) {
+    const int r = item / CW, col = (item % CW) * 4;
+    const float row_lse = fm->lse2[r];
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int p = 0; p < n; ++p) {
+      const float l = land_l[p * kRowsPerTile + r] * kLog2e;
+      const float w = (l == -INFINITY || row_lse == -INFINITY) ? 0.f : ex2(l - row_lse);
+      const float4 v = *reinterpret_cast<const float4 *>(land_o + (p * rows + r) * D + col);
+      acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
+    }
+    const int m = rt * kRowsPerTile + r, t = m / a.G, g = m % a.G;
+    const size_t e = ((size_t)(q0 + t) * a.Hq + (size_t)h * a.G + g) * D + col;
+    if (a.out_f32)
+      *reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.out) + e) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    else
+      *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(a.out) + e) =
+          make_uint2(pack2<kBf16>(acc[0], acc[1]), pack2<kBf16>(acc[2], acc[3]));
+  }
+}
 
 // ---------------------------------------------------------------------------
 // Producer warp
@@ -649,6 +702,11 @@ __device__ void math_warps(const DecodeArgs &a, uint8_t *smem, int warp, int lan
       if (warp == 0 && lane == 0) jobs[j].seg.kind = -1;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_addr(smem, D, B_JOBFULL(j)));
+      // Then join the second pass of the CTA's final merge, if the epilogue
+      // warp posts one (it lands the pieces and finds the rows' LSEs).
+      if (!warp_wait_bounded_idle(bar_addr(smem, D, B_FINAL), 0, &g_mxa_err, kErrWaitQ, lane)) return;
+      const FinalMerge *fm = reinterpret_cast<const FinalMerge *>(smem + smem_final_off(D));
+      if (fm->valid) merge_pass2_coop<D, kBf16>(a, fm, smem, warp, lane);
       return;
     }
     const int rows = tile_rows(a, qn, rt);
@@ -976,11 +1034,15 @@ constexpr uint32_t stage_land_rows() { return (uint32_t)stage_bytes(D) - 16 * kR
 // following ones.  The caller has acquired their writes (the arrival
 // count).  `own` >= 0 names a piece the caller has already placed in the
 // landing zone (rows and LSEs at its index; then all n pieces fit one
-// landing).  Returns false if a bounded wait ran out.
+// landing).  `coop`, for the unit of the CTA's last job, is where to post
+// the second pass to the math warps, which then share it
+// (merge_pass2_coop) when every piece fits one landing; `posted` tells the
+// caller that it was posted.  Returns false if a bounded wait ran out.
 template <int D, bool kBf16, int NR>
 __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int rows, int unit, int lane,
                              uint8_t *smem, uint32_t ostage, uint32_t land, uint32_t land_rows,
-                             uint32_t mbar, uint32_t &mk, int own, int lse_slots) {
+                             uint32_t mbar, uint32_t &mk, int own, int lse_slots, FinalMerge *coop,
+                             bool &posted) {
   constexpr int VEC = D / 32;
   constexpr float kLog2e = 1.4426950408889634f;
   const int n = sg.n_pieces, cf = sg.c_first;
@@ -1055,6 +1117,25 @@ __device__ bool merge_pieces(const DecodeArgs &a, const SegmentDesc &sg, int row
   if (r1 < rows && j1 == 0 && a.lse != nullptr) {
     const int mrow = sg.rt * kRowsPerTile + r1, t = mrow / a.G, g = mrow % a.G;
     a.lse[lse_index(a, sg.b, sg.q0, sg.h * a.G + g, t)] = lse2 * kLn2;
+  }
+  if (coop != nullptr && all_lse && n <= cap && rows * D > 32 * 4) {
+    // The CTA's final merge, with more (row, 4-column) items than one warp
+    // has lanes: the math warps, idle by now, join the second pass.
+    if (r1 < rows && j1 == 0) coop->lse2[r1] = lse2;
+    __syncwarp();
+    if (lane == 0) {
+      coop->seg = sg;
+      coop->rows = rows;
+      coop->land = land;
+      coop->land_rows = land_rows;
+      coop->valid = 1;
+      mbar_arrive(bar_addr(smem, D, B_FINAL));
+    }
+    __syncwarp();
+    posted = true;
+    merge_pass2_coop<D, kBf16>(a, coop, smem, kMathWarps, lane);
+    if (lane == 0) a.counters[unit] = 0ull;  // every piece has arrived; leave it clean
+    return true;
   }
   // With every LSE landed, the lanes that read a piece's LSE turn it into
   // its weight exp(lse_i - LSE) in place, once for all lanes.
@@ -1133,14 +1214,18 @@ template <int D, bool kBf16>
 __device__ __forceinline__ bool merge_unit(const DecodeArgs &a, const SegmentDesc &sg, int rows, int unit,
                                            int lane, uint8_t *smem, uint32_t ostage, uint32_t land,
                                            uint32_t land_rows, uint32_t mbar, uint32_t &mk, int own,
-                                           int lse_slots) {
+                                           int lse_slots, FinalMerge *coop, bool &posted) {
   if (rows <= 2)
-    return merge_pieces<D, kBf16, 2>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, mbar, mk, own, lse_slots);
+    return merge_pieces<D, kBf16, 2>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, mbar, mk, own,
+                                     lse_slots, coop, posted);
   if (rows <= 4)
-    return merge_pieces<D, kBf16, 4>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, mbar, mk, own, lse_slots);
+    return merge_pieces<D, kBf16, 4>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, mbar, mk, own,
+                                     lse_slots, coop, posted);
   if (rows <= 8)
-    return merge_pieces<D, kBf16, 8>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, mbar, mk, own, lse_slots);
-  return merge_pieces<D, kBf16, 16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, mbar, mk, own, lse_slots);
+    return merge_pieces<D, kBf16, 8>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, mbar, mk, own,
+                                     lse_slots, coop, posted);
+  return merge_pieces<D, kBf16, 16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, mbar, mk, own,
+                                    lse_slots, coop, posted);
 }
 
 template <int D, bool kBf16>
@@ -1194,16 +1279,26 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
   const uint32_t oland = ostage;  // free again once this job's own rows have been stored
   const uint32_t merge_bar = bar_addr(smem, D, B_MERGE);
   uint32_t mk = 0;  // phases of the merge barrier used so far
+  // The math warps wait, at the end of their work, to learn whether they
+  // join the second pass of this CTA's final merge; tell them once.
+  FinalMerge *fm = reinterpret_cast<FinalMerge *>(smem + smem_final_off(D));
+  bool posted = false;
+  auto post_none = [&]() {
+    if (!posted && lane == 0) mbar_arrive(bar_addr(smem, D, B_FINAL));  // valid stays 0
+    posted = true;
+  };
   for (int jn = 0;; ++jn) {
     const int j = jn % kJobs, jk = jn / kJobs;
     // Leaving: bulk stores this warp issued must be done with shared memory
     // (and complete) before the CTA exits.
     if (!warp_wait_bounded(bar_addr(smem, D, B_JOBFULL(j)), jk & 1, &g_mxa_err, kErrWaitFull, lane)) {
+      post_none();
       if (lane == 0) bulk_wait_all();
       return;
     }
     const SegmentDesc sg = jobs[j].seg;
     if (sg.kind < 0) {
+      post_none();
       if (lane == 0) bulk_wait_all();
       return;
     }
@@ -1357,9 +1452,10 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
       // piece's rows and LSEs (written by the async proxy, completed and
       // fenced first); the acquire lets the last piece read everyone's.
       bool ok = true;
+      FinalMerge *coop = sg.last ? fm : nullptr;
       if (merge_now) {
         ok = merge_unit<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, merge_bar, mk, own,
-                                    lse_slots);
+                                    lse_slots, coop, posted);
       } else {
         unsigned long long old = 0;
         if (lane == 0) {
@@ -1370,7 +1466,7 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
         old = __shfl_sync(0xffffffffu, old, 0);
         if ((int)(old & 0xffffffffull) + 1 == sg.n_pieces)
           ok = merge_unit<D, kBf16>(a, sg, rows, unit, lane, smem, ostage, land, land_rows, merge_bar, mk, -1,
-                                      lse_slots);
+                                      lse_slots, coop, posted);
       }
       if (hold) {
         fence_proxy_async_smem();  // reads of the landing zone precede the stage's next TMA loads
@@ -1378,6 +1474,7 @@ __device__ void epilogue_warp(const DecodeArgs &a, uint8_t *smem, int lane) {
         if (lane == 0) mbar_arrive_cnt(bar_addr(smem, D, B_EMPTY(stage)), kMathWarps);
       }
       if (!ok) {
+        post_none();
         if (lane == 0) bulk_wait_all();
         return;
       }
@@ -1410,6 +1507,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(D))
     }
     mbar_init(bar_addr(smem, D, B_MERGE), 1);
     mbar_init(bar_addr(smem, D, B_INIT), 1);
+    mbar_init(bar_addr(smem, D, B_FINAL), 1);
+    reinterpret_cast<FinalMerge *>(smem + smem_final_off(D))->valid = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -1457,6 +1556,8 @@ __global__ void __launch_bounds__(128)
   for (int d = lane * 4; d < D; d += 128) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (L != -INFINITY) {
+      // the splits' loads are independent: keep several in flight
+#pragma unroll 8
       for (int s = 0; s < S; ++s) {
         const float wgt = expf(lse_part[(size_t)s * rows + li] - L);
         const float4 v = *reinterpret_cast<const float4 *>(o_part + ((size_t)s * rows + row) * D + d);
@@ -1500,7 +1601,11 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // 3-D map {D, Hkv, pool tokens} of a K or V pool; box {64 elements, 1 head,
-// box_tokens tokens}, 128-byte swizzle, zero fill out of bounds.
+// box_tokens tokens}, 128-byte swizzle, zero fill out of bounds.  L2 fills
+// are promoted to whole rows of one head: 256 bytes for D >= 128 (the
+// second 64-column box of a row then hits), 128 bytes for D = 64, whose
+// 128-byte row a 256-byte fill would widen into the next head's row, read
+// from DRAM a second time by the CTA of that head once L2 has let it go.
 bool encode_kv_map(CUtensorMap *m, const void *base, int D, int Hkv, long long pool_tokens,
                    int box_tokens, bool bf16) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
@@ -1511,7 +1616,8 @@ bool encode_kv_map(CUtensorMap *m, const void *base, int D, int Hkv, long long p
   cuuint32_t estride[3] = {1u, 1u, 1u};
   CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                    const_cast<void *>(base), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_SWIZZLE_128B,
+                   D >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

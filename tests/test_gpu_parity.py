@@ -414,7 +414,7 @@ def test_head_dim_256_balanced_grids(grid):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("name,grid", [("ragged_varlen", 296), ("gqa_decode", 296), ("spec_mtp_small_q", 296),
-                                       ("gqa_decode_hd256", 148)])
+                                       ("long_context_split_kv", 296), ("gqa_decode_hd256", 148)])
 def test_repeated_calls_on_a_garbage_workspace(name, grid):
     # 200 calls in a row, each on a workspace whose every byte is 0xFF (NaN
     # partial results, all-ones arrival counters): every call must match the
@@ -441,3 +441,32 @@ def test_repeated_calls_on_a_garbage_workspace(name, grid):
     torch.cuda.synchronize()
     assert mxa.mxa_device_error(True) == mxa.MXA_OK
     assert worst.item() <= 2e-3, f"worst |err| over 200 calls: {worst.item():.3e}"
+
+
+@pytest.mark.parametrize("name,grid", [("ragged_varlen", 296), ("long_context_split_kv", 296), ("gqa_decode", 1000),
+                                       ("spec_mtp_small_q", 296)])
+def test_results_do_not_depend_on_which_piece_merges(name, grid):
+    # A split unit is merged by whichever of its pieces arrives last, or by a
+    # piece that finds all the others already there and merges at once,
+    # without storing its own rows.  Which piece that is, and where the
+    # pieces land (the staging buffer, a ring stage, the whole ring), changes
+    # from call to call.  The arithmetic is the same in every case and in the
+    # same order, so every call returns the same output and LSE, bit for bit.
+    w = workload(name)
+    inp = make_inputs(w)
+    q, k, v, bt, sl = to_dev(inp)
+    params = mxa.params_for(q, k, bt, inp.max_seqlen_k)
+    plan = mxa.mxa_plan_balanced(params, grid)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    lse = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device="cuda")
+    mxa.mxa_decode_fwd_f32out(q, k, v, bt, sl, params, w.scale, w.causal, plan, ws, out, lse)
+    out0, lse0 = out.clone(), lse.clone()
+    differ = torch.zeros((), dtype=torch.int64, device="cuda")
+    for _ in range(100):
+        mxa.mxa_decode_fwd_f32out(q, k, v, bt, sl, params, w.scale, w.causal, plan, ws, out, lse)
+        differ += (out.view(torch.int32) != out0.view(torch.int32)).sum()
+        differ += (lse.view(torch.int32) != lse0.view(torch.int32)).sum()
+    torch.cuda.synchronize()
+    assert mxa.mxa_device_error(True) == mxa.MXA_OK
+    assert differ.item() == 0, f"{differ.item()} values differ from the first call's over 100 calls"
