@@ -203,9 +203,8 @@ mxa_status_t mxa_plan(const mxa_decode_params_t *p, int num_splits, int sm_count
       long long cap = units * (max_blocks + 3) / 4;
       if (cap < 1) cap = 1;
       out.schedule = MXA_SCHED_BALANCED;
-      // one block per two packed rows, but no more than 6: a 16-row unit's
-      // fixed work measures at 6 blocks on B200 once its merges are cheap
-      out.unit_cost = unit_cost_for_rows(rows) < 6 ? unit_cost_for_rows(rows) : 6;
+      const int cost = unit_cost_for_rows(rows, p->D);
+      out.unit_cost = cost < max_unit_cost(p->D) ? cost : max_unit_cost(p->D);
       out.grid = (int)(slots < cap ? slots : cap);
       out.num_splits = units > 0 ? (int)ceil_div_ll(out.grid, units) : 1;
     } else {

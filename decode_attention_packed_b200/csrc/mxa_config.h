@@ -35,8 +35,15 @@ constexpr int kErrInputMask = kErrBadPage | kErrBadLen | kErrBadOffsets;
 // Fixed cost of a unit in the balanced schedule, in KV blocks: the work a
 // unit needs besides streaming its keys (the cross-warp merge, the output
 // staging and stores, the arrival and merge of a split unit) grows with its
-// packed query rows, and measures at about one block per two rows on B200.
-constexpr int unit_cost_for_rows(int rows) { return rows > 2 ? (rows + 1) / 2 : 1; }
+// packed query rows, and measures at about one 32 KiB stage of streaming per
+// two rows on B200: one block per two rows for D <= 128, one per four rows
+// for D = 256, whose blocks are 64 KiB.
+constexpr int unit_cost_for_rows(int rows, int D) {
+  return D > 128 ? (rows > 4 ? (rows + 3) / 4 : 1) : (rows > 2 ? (rows + 1) / 2 : 1);
+}
+// ... and no more than 6 blocks of 32 KiB (3 of 64 KiB): a 16-row unit's
+// fixed work measures at that once its merges are cheap.
+constexpr int max_unit_cost(int D) { return D > 128 ? 3 : 6; }
 
 // KV tokens per pipeline stage.  For D <= 128 every stage carries T x D
 // elements of K and of V (16 KiB each in 16-bit types), so T = 8192 / D:

@@ -119,7 +119,9 @@ typedef struct {
   int needs_combine;     /* 1 if units may be split across CTAs and merged (needs the workspace) */
   int unit_cost;         /* BALANCED: fixed cost of a unit, in KV blocks, added to its blocks
                             when the work is divided (0..64; mxa_plan sets one block per two
-                            packed query rows, at least 1 and at most 6); UNIFORM: unused */
+                            packed query rows, at least 1 and at most 6, and for D = 256,
+                            whose blocks are twice as large, one per four rows, at most 3);
+                            UNIFORM: unused */
   size_t workspace_bytes;/* device scratch the run needs (0 if none) */
 } mxa_plan_t;
 

@@ -124,6 +124,10 @@ def test_plan_long_context_split():
     costs = {(q, hq): mxa.mxa_plan(params(q_len=q, Hq=hq), 0, sm_count=148).unit_cost
              for q, hq in [(1, 8), (1, 16), (1, 32), (4, 32), (8, 64)]}
     assert costs == {(1, 8): 1, (1, 16): 1, (1, 32): 2, (4, 32): 6, (8, 64): 6}
+    # a D = 256 block carries twice the bytes, so the same work is half the blocks
+    costs = {(q, hq): mxa.mxa_plan(params(q_len=q, Hq=hq, D=256), 0, sm_count=148).unit_cost
+             for q, hq in [(1, 16), (1, 32), (2, 32), (4, 32)]}
+    assert costs == {(1, 16): 1, (1, 32): 1, (2, 32): 2, (4, 32): 3}
 
 
 def test_plan_does_not_split_tiny_problems():
