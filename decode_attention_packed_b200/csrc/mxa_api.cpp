@@ -85,7 +85,7 @@ mxa_status_t prepare_decode(const void *q, const void *k_cache, const void *v_ca
   mxa_plan_t use = *plan;
   if (use.schedule != MXA_SCHED_UNIFORM && use.schedule != MXA_SCHED_BALANCED) return MXA_ERR_INVALID_ARG;
   if (use.grid < 1 || use.num_splits < 1) return MXA_ERR_INVALID_ARG;
-  if (use.schedule == MXA_SCHED_BALANCED && (use.unit_cost < 0 || use.unit_cost > kMaxUnitCost))
+  if (use.schedule == MXA_SCHED_BALANCED && (use.unit_cost < 0 || use.unit_cost > kUnitCostScale * kMaxUnitCost))
     return MXA_ERR_INVALID_ARG;
   if (use.schedule == MXA_SCHED_UNIFORM) use.unit_cost = 0;
   finish_plan(p, &use);
@@ -312,7 +312,8 @@ mxa_status_t mxa_decode_fwd_varlen(const void *q, const int32_t *cu_seqlens_q, i
   // the balanced prologue sums positions of one KV head's tiles per row in 32 bits
   const long long G = p->Hq / p->Hkv;
   const long long RT = ceil_div_ll((long long)p->q_len * G, kRowsPerTile);
-  const long long row_max = RT * (ceil_div_ll(p->max_seqlen_k, block_tokens(p->D)) + L.plan.unit_cost);
+  const long long row_max =
+      RT * (ceil_div_ll(p->max_seqlen_k, block_tokens(p->D)) + ceil_div_ll(L.plan.unit_cost, kUnitCostScale));
   if (L.plan.schedule == MXA_SCHED_BALANCED && (long long)p->B * row_max > INT32_MAX) return MXA_ERR_UNSUPPORTED;
   L.cu_q = cu_seqlens_q;
   L.total_q = total_q;

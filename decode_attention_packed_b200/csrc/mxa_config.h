@@ -16,7 +16,7 @@ constexpr int kSmemPerSm = 228 * 1024;                  // B200 shared memory pe
 constexpr int kSmemReservedPerCta = 1024;               // driver-reserved shared memory per CTA
 constexpr int kMaxThreadsPerSm = 2048;
 constexpr int kMaxBalancedRows = 12288;                 // balanced schedule scans B rows in smem
-constexpr int kMaxUnitCost = 64;
+constexpr int kMaxUnitCost = 64;                       // blocks; unit_cost <= 4 x this
 
 // Device-side failure record (bit flags), read back by mxa_device_error():
 // bounded waits that ran out and a misaligned shared-memory base (reported
@@ -32,18 +32,21 @@ enum : int {
 };
 constexpr int kErrInputMask = kErrBadPage | kErrBadLen | kErrBadOffsets;
 
-// Fixed cost of a unit in the balanced schedule, in KV blocks: the work a
-// unit needs besides streaming its keys (the cross-warp merge, the output
-// staging and stores, the arrival and merge of a split unit) grows with its
-// packed query rows, and measures at about one 32 KiB stage of streaming per
-// two rows on B200: one block per two rows for D <= 128, one per four rows
-// for D = 256, whose blocks are 64 KiB.
+// Fixed cost of a unit in the balanced schedule, in quarter KV blocks (the
+// plan's unit_cost): the work a unit needs besides streaming its keys (the
+// cross-warp merge, the output staging and stores, the arrival and merge of
+// a split unit) grows with its packed query rows.  Measured on B200 (sweeps
+// per workload): one 32 KiB block for one or two rows, a block and a half
+// for three or four, one block per two rows above that (D <= 128); one
+// 64 KiB block per four rows for D = 256.
+constexpr int kUnitCostScale = 4;  // unit_cost counts quarter blocks
 constexpr int unit_cost_for_rows(int rows, int D) {
-  return D > 128 ? (rows > 4 ? (rows + 3) / 4 : 1) : (rows > 2 ? (rows + 1) / 2 : 1);
+  return D > 128 ? kUnitCostScale * (rows > 4 ? (rows + 3) / 4 : 1)
+                 : (rows <= 2 ? kUnitCostScale : rows <= 4 ? kUnitCostScale * 3 / 2 : kUnitCostScale * ((rows + 1) / 2));
 }
 // ... and no more than 6 blocks of 32 KiB (3 of 64 KiB): a 16-row unit's
 // fixed work measures at that once its merges are cheap.
-constexpr int max_unit_cost(int D) { return D > 128 ? 3 : 6; }
+constexpr int max_unit_cost(int D) { return kUnitCostScale * (D > 128 ? 3 : 6); }
 
 // KV tokens per pipeline stage.  For D <= 128 every stage carries T x D
 // elements of K and of V (16 KiB each in 16-bit types), so T = 8192 / D:

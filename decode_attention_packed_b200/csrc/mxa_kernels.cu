@@ -121,14 +121,23 @@ __device__ void merge_pass2_coop(const DecodeArgs &a, const FinalMerge *fm, cons
 // Producer warp
 // ---------------------------------------------------------------------------
 
+// Fixed cost, in KV blocks, of each unit of batch row i: the plan's unit
+// cost is in quarter blocks, and the rows share it out in whole blocks
+// (row i gets floor((i + 1) q / 4) - floor(i q / 4)), so a cost below one
+// block still weighs what it should over a range of many short rows.
+__device__ __forceinline__ int row_cost(const DecodeArgs &a, int i) {
+  return (int)(((long long)(i + 1) * a.unit_cost) / kUnitCostScale - ((long long)i * a.unit_cost) / kUnitCostScale);
+}
+
 // Cursor over this CTA's range of work.  BALANCED: positions in a
 // flattened cost space in which every unit (batch row b with nb > 0 KV
-// blocks, KV head x row tile hr) spans unit_cost + nb positions: first its
-// fixed cost, then one position per KV block.  `x` is the position of block
-// `blk` of the current unit and `end` closes the CTA's range.  UNIFORM:
-// positions are the unit's block indices.
+// blocks, KV head x row tile hr) spans V_b + nb positions: first its fixed
+// cost V_b = row_cost(b), then one position per KV block.  `x` is the
+// position of block `blk` of the current unit and `end` closes the CTA's
+// range.  UNIFORM: positions are the unit's block indices.
 struct Cursor {
   int b, hr, blk;
+  int V;              // fixed cost of each unit of row b (balanced schedule)
   long long x, end;
   long long per_cta;  // positions per CTA range (balanced schedule)
   int L, nb;          // length and blocks of row b
@@ -185,6 +194,7 @@ __device__ __forceinline__ void cursor_enter_row(Cursor &c, const DecodeArgs &a,
     c.qn = a.q_len;
   }
   c.L_next = c.b + 1 < a.B ? (long long)a.seqlens[c.b + 1] + a.len_add : 0;  // consumed a segment later
+  c.V = a.schedule == MXA_SCHED_BALANCED ? row_cost(a, c.b) : 0;
 }
 
 // The segment at the cursor (a contiguous block range of one unit); the
@@ -221,18 +231,19 @@ __device__ SegmentDesc cursor_take(Cursor &c, const DecodeArgs &a) {
     c.blk = 0;
     if (++c.hr == HR) {
       c.hr = 0;
-      if (c.x + a.unit_cost < c.end && c.b + 1 < a.B) {
+      if (c.b + 1 < a.B) {
         ++c.b;
         cursor_enter_row<D, kVarlen>(c, a, clamp_len(c.L_next, a.max_seqlen_k));
         while (c.nb == 0 && c.b + 1 < a.B) {  // rows without keys (or queries) hold no units
           ++c.b;
           cursor_enter_row<D, kVarlen>(c, a, clamp_len((long long)a.seqlens[c.b] + a.len_add, a.max_seqlen_k));
         }
+        if (c.x + c.V >= c.end) c.end = c.x;  // that unit's first block lies past this range
       } else {
         c.end = c.x;
       }
     }
-    c.x += a.unit_cost;  // the next unit's first block follows its fixed cost
+    c.x += c.V;  // the next unit's first block follows its fixed cost
   }
   return s;
 }
@@ -250,10 +261,10 @@ template <int D, bool kVarlen>
 __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cursor &tail, bool &has_tail) {
   constexpr int T = block_tokens(D);
   const int HR = a.Hkv * a.RT;
-  const int V = a.unit_cost;
   Cursor c;
   c.hr = 0;
   c.blk = 0;
+  c.V = 0;
   c.x = c.end = 0;
   c.per_cta = 1;
   c.L = c.nb = c.L_next = 0;
@@ -285,7 +296,7 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
     const int L = clamp_len((long long)a.seqlens[i] + a.len_add, a.max_seqlen_k);
     lens[i] = L;
     const int nb = (L + T - 1) / T;
-    int w = nb > 0 ? nb + V : 0;  // positions of one unit of row i
+    int w = nb > 0 ? nb + row_cost(a, i) : 0;  // positions of one unit of row i
     if constexpr (kVarlen) {      // times the row's tiles: one KV head's units
       int q0, qn;
       row_queries<true>(a, i, q0, qn);
@@ -323,6 +334,8 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
     const long long pre = lo_b > 0 ? scan[lo_b - 1] : 0;
     const long long w = scan[lo_b] - pre;  // > 0: the row holds position x0
     const long long off = x0 - HS * pre;
+    const int V = row_cost(a, lo_b);
+    c.V = V;
     // positions of one unit of the row (from the scan, or its length)
     const long long uw = kVarlen ? (long long)((lens[lo_b] + T - 1) / T + V) : w;
     const long long pos = off % uw;
@@ -356,13 +369,15 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
     const long long pre_l = lb > 0 ? scan[lb - 1] : 0;
     const long long w_l = scan[lb] - pre_l;
     const long long off_l = xl - HS * pre_l;
-    const long long uw_l = kVarlen ? (long long)((lens[lb] + T - 1) / T + V) : w_l;
+    const int Vl = row_cost(a, lb);
+    const long long uw_l = kVarlen ? (long long)((lens[lb] + T - 1) / T + Vl) : w_l;
     const long long pos_l = off_l % uw_l;
-    if (pos_l >= V) {  // xl falls on a KV block of that unit
-      const int nb_l = (int)(uw_l - V), blk_l = (int)(pos_l - V);
+    if (pos_l >= Vl) {  // xl falls on a KV block of that unit
+      const int nb_l = (int)(uw_l - Vl), blk_l = (int)(pos_l - Vl);
       const long long x_t = xl - blk_l;  // position of that unit's first block
-      if (blk_l + 1 < nb_l && x_t - V > x0) {
+      if (blk_l + 1 < nb_l && x_t - Vl > x0) {
         tail.b = lb;
+        tail.V = Vl;
         tail.hr = (int)(off_l / uw_l);
         tail.blk = 0;
         tail.x = x_t;
@@ -379,7 +394,7 @@ __device__ Cursor cursor_start(const DecodeArgs &a, uint8_t *smem, int lane, Cur
           tail.qn = a.q_len;
         }
         has_tail = true;
-        c.end = x_t - V;  // the main walk stops where that unit begins
+        c.end = x_t - Vl;  // the main walk stops where that unit begins
       }
     }
   }

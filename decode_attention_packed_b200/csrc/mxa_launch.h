@@ -41,7 +41,7 @@ struct DecodeArgs {
   int splits;                  // UNIFORM: splits per unit
   int chunk_blocks;            // UNIFORM: blocks per split
   int units;
-  int unit_cost;               // BALANCED: fixed cost of a unit, in KV blocks
+  int unit_cost;               // BALANCED: fixed cost of a unit, in quarter KV blocks
   int len_add;                 // new tokens appended to each row this call (0: none)
   const uint16_t *k_new;       // [B, q_len, Hkv, D]: the appended tokens' keys (len_add > 0)
   const uint16_t *v_new;       //   and values

@@ -69,10 +69,11 @@ typedef enum { MXA_F16 = 0, MXA_BF16 = 1 } mxa_dtype_t;
  * BALANCED: the work of all units, laid end to end (unit-major), is
  *           divided into `grid` equal contiguous ranges, one per CTA; a unit
  *           that straddles ranges is merged by the combine pass.  A unit's
- *           work is its KV blocks plus a fixed cost of `unit_cost` blocks
- *           (its query load, the merge of its warps' results and its output
- *           stores), so every CTA gets the same work however ragged the
- *           lengths are (a length-aware split in the spirit of the
+ *           work is its KV blocks plus a fixed cost of `unit_cost` quarter
+ *           blocks (its query load, the merge of its warps' results and its
+ *           output stores; a cost below a whole block is shared out over the
+ *           rows in whole blocks), so every CTA gets the same work however
+ *           ragged the lengths are (a length-aware split in the spirit of the
  *           cost-balanced core assignment of "MixedQuantSparseFlashMlaMetadata
  *           算子解析", section 源码级原理, which also charges each task a fixed
  *           cost besides its KV length). */
@@ -117,10 +118,11 @@ typedef struct {
   int ctas_per_sm;       /* resident CTAs per SM the plan assumed: 2, or 1 for D = 256 */
   int sm_count;          /* SMs the plan assumed */
   int needs_combine;     /* 1 if units may be split across CTAs and merged (needs the workspace) */
-  int unit_cost;         /* BALANCED: fixed cost of a unit, in KV blocks, added to its blocks
-                            when the work is divided (0..64; mxa_plan sets one block per two
-                            packed query rows, at least 1 and at most 6, and for D = 256,
-                            whose blocks are twice as large, one per four rows, at most 3);
+  int unit_cost;         /* BALANCED: fixed cost of a unit, in QUARTER KV blocks, added to
+                            its blocks when the work is divided (0..256; mxa_plan sets half
+                            a block for units of one or two packed query rows, else one
+                            block per two rows, at most 6 blocks; for D = 256, whose blocks
+                            are twice as large, one per four rows, at least 1, at most 3);
                             UNIFORM: unused */
   size_t workspace_bytes;/* device scratch the run needs (0 if none) */
 } mxa_plan_t;
@@ -220,7 +222,7 @@ MXA_API mxa_status_t mxa_decode_fwd(const void *q, const void *k_cache, const vo
 /* As mxa_decode_fwd, but run a plan the caller resolved (or built) before:
  * the second phase of the two-phase call.  The plan is validated against
  * `params` (schedule, grid >= 1, units, block_tokens); a BALANCED plan may
- * use any grid >= 1 and any unit_cost in 0..64. */
+ * use any grid >= 1 and any unit_cost in 0..256 (quarter blocks). */
 MXA_API mxa_status_t mxa_decode_fwd_with_plan(const void *q, const void *k_cache, const void *v_cache,
                                       const int32_t *block_table, const int32_t *cache_seqlens,
                                       const mxa_decode_params_t *params, float scale, int causal,

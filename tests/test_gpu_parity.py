@@ -108,11 +108,12 @@ def test_ragged_balanced_grids(grid):
     check(inp, out, lse, ref)
 
 
-@pytest.mark.parametrize("unit_cost", [0, 1, 5, 64])
+@pytest.mark.parametrize("unit_cost", [0, 1, 2, 5, 64, 256])
 @pytest.mark.parametrize("grid", [3, 296, 1500])
 def test_balanced_unit_costs(grid, unit_cost):
-    # the fixed cost per unit moves every range boundary; every block must
-    # still be read exactly once and every split unit merged
+    # the fixed cost per unit (quarter blocks, shared out over the rows in
+    # whole blocks) moves every range boundary; every block must still be
+    # read exactly once and every split unit merged
     inp, ref, dev = full(4)
     q, k, v, bt, sl = dev
     plan = mxa.mxa_plan_balanced(mxa.params_for(q, k, bt, inp.max_seqlen_k), grid)
@@ -121,7 +122,7 @@ def test_balanced_unit_costs(grid, unit_cost):
     check(inp, out, lse, ref)
 
 
-@pytest.mark.parametrize("unit_cost", [0, 3, 64])
+@pytest.mark.parametrize("unit_cost", [0, 3, 6, 64, 256])
 def test_balanced_unit_costs_edge_lengths(unit_cost):
     # rows of every length class, including L = 0 rows that hold no unit
     inp = make_inputs(wl())

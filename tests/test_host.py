@@ -116,18 +116,19 @@ def test_plan_long_context_split():
     assert plan.units == 16 and plan.grid == 296 and plan.num_splits == 19
     assert plan.ctas_per_sm == 2 and plan.block_tokens == 64
     assert plan.needs_combine == 1 and plan.workspace_bytes > 0
-    # each unit is charged a fixed cost besides its KV blocks: one block per
-    # two packed query rows (8 rows here), at least one and at most six
-    assert plan.unit_cost == 4
-    assert mxa.mxa_plan_balanced(params(), 100, sm_count=148).unit_cost == 4
+    # each unit is charged a fixed cost besides its KV blocks, in quarter
+    # blocks: one block per two packed query rows (8 rows here), one block for
+    # one or two rows, a block and a half for three or four, at most six
+    assert plan.unit_cost == 16
+    assert mxa.mxa_plan_balanced(params(), 100, sm_count=148).unit_cost == 16
     assert mxa.mxa_plan(params(), 3, sm_count=148).unit_cost == 0
     costs = {(q, hq): mxa.mxa_plan(params(q_len=q, Hq=hq), 0, sm_count=148).unit_cost
              for q, hq in [(1, 8), (1, 16), (1, 32), (4, 32), (8, 64)]}
-    assert costs == {(1, 8): 1, (1, 16): 1, (1, 32): 2, (4, 32): 6, (8, 64): 6}
+    assert costs == {(1, 8): 4, (1, 16): 4, (1, 32): 6, (4, 32): 24, (8, 64): 24}
     # a D = 256 block carries twice the bytes, so the same work is half the blocks
     costs = {(q, hq): mxa.mxa_plan(params(q_len=q, Hq=hq, D=256), 0, sm_count=148).unit_cost
              for q, hq in [(1, 16), (1, 32), (2, 32), (4, 32)]}
-    assert costs == {(1, 16): 1, (1, 32): 1, (2, 32): 2, (4, 32): 3}
+    assert costs == {(1, 16): 4, (1, 32): 4, (2, 32): 8, (4, 32): 12}
 
 
 def test_plan_does_not_split_tiny_problems():
@@ -231,8 +232,8 @@ def test_run_refuses_bad_arguments_before_launch():
     bad = mxa.mxa_plan(p, 2, sm_count=148)
     bad.grid += 1
     assert _run_with_plan(p, bad, ws=1, ws_bytes=1 << 30) == MXA_ERR_INVALID_ARG
-    # a balanced plan's fixed unit cost must lie in 0..64
-    for cost in (-1, 65):
+    # a balanced plan's fixed unit cost must lie in 0..256 quarter blocks
+    for cost in (-1, 257):
         bad = mxa.mxa_plan(p, 0, sm_count=148)
         bad.unit_cost = cost
         assert _run_with_plan(p, bad, ws=1, ws_bytes=1 << 30) == MXA_ERR_INVALID_ARG
@@ -293,7 +294,7 @@ def test_varlen_refuses_bad_arguments_before_launch():
     big = params(B=1000, q_len=2, Hq=16, Hkv=1, D=128, page_size=64, num_pages=16,
                  max_pages_per_seq=1073700, max_seqlen_k=1073700 * 64)
     bplan = mxa.mxa_plan_balanced(big, 296, sm_count=148)
-    bplan.unit_cost = 64
+    bplan.unit_cost = 256
     assert call(p=big, plan=bplan) == mxa.MXA_ERR_UNSUPPORTED
 
 
