@@ -57,11 +57,11 @@ METRIC = "decode-attn µs/call and KV-read GB/s as % of B200 HBM peak (1 GPU)"
 # the bench reports null.  The captures and their commands are summarised
 # under profiles/ (the median of three launches after five).
 MEASURED_TRAFFIC = {
-    ("a0a165d28fc62be4", "ragged_varlen"): 518_806_016,
-    ("a0a165d28fc62be4", "gqa_decode"): 245_970_944,
-    ("a0a165d28fc62be4", "spec_mtp_small_q"): 217_385_216,
-    ("a0a165d28fc62be4", "long_context_split_kv"): 134_759_168,
-    ("a0a165d28fc62be4", "gqa_decode_hd256"): 315_080_448,
+    ("dd2bfde320a38581", "ragged_varlen"): 518_542_592,
+    ("dd2bfde320a38581", "gqa_decode"): 246_210_048,
+    ("dd2bfde320a38581", "spec_mtp_small_q"): 216_960_256,
+    ("dd2bfde320a38581", "long_context_split_kv"): 134_545_920,
+    ("dd2bfde320a38581", "gqa_decode_hd256"): 315_172_352,
 }
 HEADLINE = "ragged_varlen"
 SUITE = ("gqa_decode", "spec_mtp_small_q", "long_context_split_kv")
