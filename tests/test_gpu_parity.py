@@ -151,6 +151,21 @@ def test_one_unit_in_many_pieces(D, dtype, G, grid):
     check(inp, out, lse)
 
 
+@pytest.mark.parametrize("grid", [5, 6, 12, 13, 100, 300])
+def test_rows_of_one_length(grid):
+    # Rows all of one length: the balanced ranges then fall at the same
+    # offsets in every unit, or straddle two units, depending on the grid
+    # (6 units of 47 blocks here, over 5 to 300 CTAs).
+    w = Workload(name="even", B=3, q_len=1, Hq=8, Hkv=2, D=128, dtype="bf16", page_size=16, causal=False,
+                 lengths="const:3000", seed=93)
+    inp = make_inputs(w)
+    dev = to_dev(inp)
+    q, k, v, bt, sl = dev
+    plan = mxa.mxa_plan_balanced(mxa.params_for(q, k, bt, inp.max_seqlen_k), grid)
+    out, lse, _ = run_gpu(inp, plan=plan, dev=dev)
+    check(inp, out, lse)
+
+
 @pytest.mark.parametrize("B", [12288, 12289])
 def test_row_limit_of_the_balanced_schedule(B):
     # the largest batch the balanced prologue scans, and one row more (the
