@@ -119,11 +119,11 @@ typedef struct {
   int sm_count;          /* SMs the plan assumed */
   int needs_combine;     /* 1 if units may be split across CTAs and merged (needs the workspace) */
   int unit_cost;         /* BALANCED: fixed cost of a unit, in QUARTER KV blocks, added to
-                            its blocks when the work is divided (0..256; mxa_plan sets half
-                            a block for units of one or two packed query rows, else one
-                            block per two rows, at most 6 blocks; for D = 256, whose blocks
-                            are twice as large, one per four rows, at least 1, at most 3);
-                            UNIFORM: unused */
+                            its blocks when the work is divided (0..256; mxa_plan sets one
+                            block for units of one or two packed query rows, a block and a
+                            half for three or four, else one block per two rows, at most 6
+                            blocks; for D = 256, whose blocks are twice as large, one per
+                            four rows, at least 1, at most 3); UNIFORM: unused */
   size_t workspace_bytes;/* device scratch the run needs (0 if none) */
 } mxa_plan_t;
 
